@@ -1,0 +1,204 @@
+"""CPU oracle for the MoonEP balanced expert-parallel hot path — TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's ``cpu_baseline``
+leg may import this package.  It wraps the plain C implementation in
+``moonep_oracle.c`` (built with gcc, strict IEEE arithmetic, no fast-math) and
+shares nothing with the CUDA library: no code, header, table or constant.
+
+What each function follows, and what pins it (the ``-m "not gpu"`` tests):
+
+* ``plan`` — the pages fix the outcome: every rank receives exactly S*K
+  token-slots ("Moonshot AI Open-Sources MoonEP", S x K paragraph), overloaded
+  experts are duplicated onto other ranks within a per-rank replica-slot budget
+  (same page, replica-slot paragraph), buffers have a fixed NvS = S*K +
+  alignment padding rows ("MoonshotAI/MoonEP 딥다이브" §4 pattern 2).  The
+  tie-breaks are this build's fixed reading (see the C file header).  Pinned by:
+  a hand-derived worked example; closed-form degenerate routings (all tokens on
+  one expert, already-balanced routing); invariants on random routings (S*K
+  rows per rank, bijection pairs -> rows, row expert = routed expert, replica
+  budget, overflow/deficit accounting, piece-count bound, independence of H);
+  and an independent lexsort formulation of the keep/overflow/receiver order.
+* ``dispatch`` — the bit-copy definition (§2② zero copy); pinned by the
+  round trip and the "every row written exactly once" poison check.
+* ``combine`` — fp32 gate-weighted sum (§3③ combine); pinned against the fp64
+  closed form sum_k w_k x within the bf16 + fp32 rounding bound (§8 exercise C).
+* ``combine_backward`` — per-element closed forms: dY = w*dOut within half a bf16
+  ulp of the fp64 product; dgate = <dOut, x> for the identity expert, in fp64.
+* ``reduce_grad`` — with integer-valued bf16 gradients all fp32 sums are
+  exact, so home + replicas must equal, bit for bit, the no-replication
+  gradient (§4 pattern 3, §8 exercise E).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, Optional, Tuple
+
+import numpy as np
+
+from .build import LIB_PATH, build
+
+OK = 0
+INVALID_ARG = 1
+BAD_EXPERT_ID = 2
+BUDGET = 4
+CAPACITY = 8
+
+KIND_NATIVE = 0
+KIND_REPLICA = 1
+KIND_REMOTE = 2
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("R", "E", "K", "S", "H", "budget", "mode", "align")]
+
+    def __init__(self, R, E, K, S, H=1, budget=0, mode=0, align=1):
+        super().__init__(R, E, K, S, H, budget, mode, align)
+
+    @classmethod
+    def of(cls, w, **over) -> "Config":
+        d = dict(R=w.R, E=w.E, K=w.K, S=w.S, H=w.H, budget=w.budget, mode=w.mode,
+                 align=getattr(w, "align", 1))
+        d.update(over)
+        return cls(**d)
+
+
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_PLAN_FIELDS = ["expert_count", "rank_load", "overflow", "deficit", "n_seg", "seg_expert",
+                "seg_start", "seg_len", "seg_kind", "seg_wslot", "n_piece", "piece_expert",
+                "piece_rank", "piece_start", "piece_len", "piece_wslot", "piece_ostart",
+                "rep_expert", "n_remote", "slot_of", "slot_src"]
+
+
+class _PlanOut(ctypes.Structure):
+    _fields_ = [(n, _I32P) for n in _PLAN_FIELDS]
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        vp = ctypes.c_void_p
+        cp = ctypes.POINTER(Config)
+        lib.orc_nvs.argtypes = [cp]
+        lib.orc_nvs.restype = ctypes.c_int64
+        lib.orc_plan.argtypes = [cp, vp, ctypes.POINTER(_PlanOut)]
+        lib.orc_plan.restype = ctypes.c_int
+        lib.orc_dispatch.argtypes = [cp, vp, vp, vp]
+        lib.orc_dispatch.restype = None
+        lib.orc_combine_tokens.argtypes = [cp, vp, vp, vp, vp, ctypes.c_int64, vp]
+        lib.orc_combine_tokens.restype = None
+        lib.orc_combine_backward_tokens.argtypes = [cp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp]
+        lib.orc_combine_backward_tokens.restype = None
+        lib.orc_reduce_grad.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
+        lib.orc_reduce_grad.restype = None
+        lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.orc_f32_to_bf16.restype = ctypes.c_uint16
+        lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.orc_bf16_to_f32.restype = ctypes.c_float
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def nvs(cfg: Config) -> int:
+    return int(_L().orc_nvs(ctypes.byref(cfg)))
+
+
+def plan(cfg: Config, topk_idx: np.ndarray) -> Tuple[int, Dict[str, np.ndarray]]:
+    """Run the plan.  Returns (status, tables); tables hold the valid prefix of each."""
+    R, E, K, S, B = cfg.R, cfg.E, cfg.K, cfg.S, cfg.budget
+    n_pairs = R * S * K
+    NvS = nvs(cfg) if R > 0 and cfg.align >= 1 else 0
+    sizes = dict(expert_count=E, rank_load=R, overflow=R, deficit=R, n_seg=R, seg_expert=R * E,
+                 seg_start=R * E, seg_len=R * E, seg_kind=R * E, seg_wslot=R * E, n_piece=1,
+                 piece_expert=E + R, piece_rank=E + R, piece_start=E + R, piece_len=E + R,
+                 piece_wslot=E + R, piece_ostart=E + R, rep_expert=max(R * B, 1), n_remote=1,
+                 slot_of=max(n_pairs, 1), slot_src=max(R * NvS, 1))
+    arrs = {k: np.full(max(v, 1), -7, dtype=np.int32) for k, v in sizes.items()}
+    out = _PlanOut(**{k: a.ctypes.data_as(_I32P) for k, a in arrs.items()})
+    idx = _c(topk_idx, np.int32).ravel()
+    st = int(_L().orc_plan(ctypes.byref(cfg), _p(idx), ctypes.byref(out)))
+    arrs["slot_of"] = arrs["slot_of"][:n_pairs]
+    arrs["slot_src"] = arrs["slot_src"][:R * NvS]
+    arrs["rep_expert"] = arrs["rep_expert"][:R * B]
+    np_ = int(arrs["n_piece"][0]) if st in (OK, BUDGET) else 0
+    for k in ("piece_expert", "piece_rank", "piece_start", "piece_len", "piece_wslot",
+              "piece_ostart"):
+        arrs[k] = arrs[k][:np_]
+    for k in ("seg_expert", "seg_start", "seg_len", "seg_kind", "seg_wslot"):
+        arrs[k] = arrs[k].reshape(R, E)
+    arrs["nvs"] = np.array([NvS], np.int64)
+    return st, arrs
+
+
+def dispatch(cfg: Config, slot_of: np.ndarray, x: np.ndarray, recv: Optional[np.ndarray] = None
+             ) -> np.ndarray:
+    """recv[slot_of[p]] = x[p // K]; ``recv`` (uint16 [R*NvS, H]) is updated in place."""
+    NvS = nvs(cfg)
+    if recv is None:
+        recv = np.zeros((cfg.R * NvS, cfg.H), np.uint16)
+    s = _c(slot_of, np.int32)
+    xx = _c(x, np.uint16)
+    _L().orc_dispatch(ctypes.byref(cfg), _p(s), _p(xx), _p(recv))
+    return recv
+
+
+def combine(cfg: Config, slot_of: np.ndarray, y: np.ndarray, gates: np.ndarray,
+            tokens: Optional[np.ndarray] = None) -> np.ndarray:
+    """bf16 bits [n_tokens, H] of sum_k w_k y[slot_k] for the listed tokens (all if None)."""
+    s = _c(slot_of, np.int32)
+    g = _c(gates, np.float32)
+    yy = _c(y, np.uint16)
+    n = cfg.R * cfg.S if tokens is None else len(tokens)
+    tk = None if tokens is None else _c(tokens, np.int64)
+    out = np.zeros((n, cfg.H), np.uint16)
+    _L().orc_combine_tokens(ctypes.byref(cfg), _p(s), _p(yy), _p(g), _p(tk), n, _p(out))
+    return out
+
+
+def combine_backward(cfg: Config, slot_of: np.ndarray, dout: np.ndarray, y: np.ndarray,
+                     gates: np.ndarray, tokens: Optional[np.ndarray] = None
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """(dY rows bf16 [n_tokens, K, H], dgates fp32 [n_tokens, K]) for the listed tokens."""
+    s = _c(slot_of, np.int32)
+    g = _c(gates, np.float32)
+    d = _c(dout, np.uint16)
+    yy = _c(y, np.uint16)
+    n = cfg.R * cfg.S if tokens is None else len(tokens)
+    tk = None if tokens is None else _c(tokens, np.int64)
+    dy = np.zeros((n, cfg.K, cfg.H), np.uint16)
+    dg = np.zeros((n, cfg.K), np.float32)
+    _L().orc_combine_backward_tokens(ctypes.byref(cfg), _p(s), _p(d), _p(yy), _p(g), _p(tk), n,
+                                     _p(dy), _p(dg))
+    return dy, dg
+
+
+def reduce_grad(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray, home: np.ndarray
+                ) -> np.ndarray:
+    """New home gradients (bf16 bits [E, P]); ``rep`` is [R, budget, P]."""
+    home = np.array(home, dtype=np.uint16, copy=True, order="C")
+    rep = _c(rep, np.uint16)
+    P = home.shape[-1]
+    pe = _c(tables["piece_expert"], np.int32)
+    pr = _c(tables["piece_rank"], np.int32)
+    pw = _c(tables["piece_wslot"], np.int32)
+    _L().orc_reduce_grad(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(rep), _p(home), P)
+    return home
+
+
+def f32_to_bf16(v: float) -> int:
+    return int(_L().orc_f32_to_bf16(float(v)))
+
+
+def bf16_to_f32(b: int) -> float:
+    return float(_L().orc_bf16_to_f32(int(b)))
