@@ -1,0 +1,227 @@
+"""GPU dispatch / combine / combine-backward / reduce_grad vs the CPU oracle.
+
+Bar: dispatched rows bit-exact (and padding rows untouched); combine,
+combine-backward and reduce_grad within 1e-3 norm-relative error
+(max |gpu - ref| / max |ref|) with fp32 accumulation.  The bit-identical
+fraction is also asserted where both sides round the same fp32 value.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from moonep_inputs import (WORKLOADS, bf16_bits_to_f32, integer_bf16, make_gates, make_routing,
+                           make_x, normal_bf16, uniform_routing)
+from tests.gpu_util import POISON, configs, gpu_plan, rel_err, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+
+
+def _setup(R, E, K, S, H, mv=3.0, seed=0, budget=None, mode=0, align=1):
+    cfg, ocfg = configs(R, E, K, S, H=H, budget=budget, mode=mode, align=align)
+    if S == 0:
+        idx = np.zeros((R, 0, K), np.int32)
+    elif E > K:
+        idx, _, _ = make_routing(R, E, K, S, mv, seed=seed)
+    else:
+        idx = uniform_routing(R, E, K, S, seed=seed)
+    ost, ot = oracle.plan(ocfg, idx)
+    gst, arena, gv, _ = gpu_plan(cfg, idx)
+    assert np.array_equal(gv["slot_of"], ot["slot_of"])
+    return cfg, ocfg, ot, arena
+
+
+def _dispatch(cfg, arena, x_np, NvS, offset_elems=0):
+    """Run dispatch into a poisoned buffer; offset_elems shifts the buffers (alignment tests)."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    H = cfg.H
+    nrows = cfg.R * NvS
+    xs = to_dev(np.concatenate([np.zeros(offset_elems, np.uint16), x_np.ravel()]))
+    x = xs[offset_elems:]
+    rb = torch.full((nrows * H + offset_elems,), POISON - 65536,
+                    dtype=torch.int16, device=x.device)
+    recv = rb[offset_elems:]
+    status = torch.zeros(1, dtype=torch.int32, device=x.device)
+    me.moonep_dispatch(cfg, arena, x, recv, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return to_np(recv).reshape(nrows, H)
+
+
+SHAPES = [
+    # R, E, K, S, H, align
+    (8, 32, 4, 256, 512, 1),     # the small parity workload
+    (2, 4, 2, 9, 24, 1),
+    (4, 16, 8, 33, 136, 16),
+    (3, 9, 3, 17, 13, 4),        # H not a multiple of 8: scalar path
+    (1, 4, 2, 5, 8, 1),
+    (8, 64, 6, 40, 1, 1),        # H = 1
+    (4, 16, 2, 0, 64, 1),        # empty batch
+    (8, 64, 8, 1200, 1032, 1),   # several blocks, ragged vector tail (129 vectors per row)
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_dispatch_bitwise(shape):
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A)
+    NvS = int(ot["nvs"][0])
+    x = make_x(R, S, H, seed=1).reshape(R * S, H)
+    got = _dispatch(cfg, arena, x, NvS)
+    ref = oracle.dispatch(ocfg, ot["slot_of"], x,
+                          np.full((R * NvS, H), POISON, np.uint16))
+    assert np.array_equal(got, ref)
+    # every valid row written exactly once with its source row, padding untouched
+    valid = ot["slot_src"] >= 0
+    assert (got[~valid] == POISON).all()
+
+
+def test_dispatch_misaligned_buffers_take_the_scalar_path():
+    cfg, ocfg, ot, arena = _setup(4, 16, 4, 20, 64)
+    NvS = int(ot["nvs"][0])
+    x = make_x(4, 20, 64, seed=2).reshape(80, 64)
+    got = _dispatch(cfg, arena, x, NvS, offset_elems=1)
+    ref = oracle.dispatch(ocfg, ot["slot_of"], x, np.full((4 * NvS, 64), POISON, np.uint16))
+    assert np.array_equal(got, ref)
+
+
+def _combine(cfg, arena, y_np, w_np):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    y = to_dev(y_np)
+    w = to_dev(w_np.astype(np.float32).ravel())
+    out = torch.empty((cfg.R * cfg.S, cfg.H), dtype=torch.int16, device=y.device)
+    status = torch.zeros(1, dtype=torch.int32, device=y.device)
+    me.moonep_combine(cfg, arena, y, w, out, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return to_np(out)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_combine_matches_oracle(shape):
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A, seed=3)
+    NvS = int(ot["nvs"][0])
+    y = normal_bf16((R * NvS, H), seed=3, stream=9)
+    w = make_gates(R, S, K, seed=3)
+    got = _combine(cfg, arena, y, w)
+    ref = oracle.combine(ocfg, ot["slot_of"], y, w)
+    if ref.size == 0:
+        assert got.size == 0
+        return
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999
+
+
+@pytest.mark.parametrize("shape", SHAPES[:3])
+def test_round_trip_identity_expert(shape):
+    """dispatch -> identity expert -> combine == sum_k w_k x (§8 exercise C)."""
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A, seed=4)
+    NvS = int(ot["nvs"][0])
+    x = make_x(R, S, H, seed=4).reshape(R * S, H)
+    recv = _dispatch(cfg, arena, x, NvS)
+    w = make_gates(R, S, K, seed=4)
+    got = _combine(cfg, arena, recv, w)
+    ref = oracle.combine(ocfg, ot["slot_of"], oracle.dispatch(ocfg, ot["slot_of"], x), w)
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    exact = w.reshape(R * S, K).astype(np.float64).sum(1, keepdims=True) * bf16_bits_to_f32(x)
+    assert rel_err(bf16_bits_to_f32(got), exact) <= 2 ** -7
+
+
+def _combine_bwd(cfg, arena, dout_np, y_np, w_np, NvS):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    dout = to_dev(dout_np)
+    y = to_dev(y_np)
+    w = to_dev(w_np.astype(np.float32).ravel())
+    dy = torch.full((cfg.R * NvS, cfg.H), POISON - 65536,
+                    dtype=torch.int16, device=y.device)
+    dg = torch.full((cfg.R * cfg.S * cfg.K,), float("nan"), dtype=torch.float32, device=y.device)
+    status = torch.zeros(1, dtype=torch.int32, device=y.device)
+    me.moonep_combine_backward(cfg, arena, dout, y, w, dy, dg, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return to_np(dy), to_np(dg)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_combine_backward_matches_oracle(shape):
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A, seed=5)
+    NvS = int(ot["nvs"][0])
+    y = normal_bf16((R * NvS, H), seed=5, stream=9)
+    dout = normal_bf16((R * S, H), seed=5, stream=3)
+    w = make_gates(R, S, K, seed=5)
+    dy, dg = _combine_bwd(cfg, arena, dout, y, w, NvS)
+    ref_dy, ref_dg = oracle.combine_backward(ocfg, ot["slot_of"], dout, y, w)
+    if R * S == 0:
+        return
+    so = ot["slot_of"]
+    got_rows = dy[so].reshape(R * S, K, H)
+    assert rel_err(bf16_bits_to_f32(got_rows), bf16_bits_to_f32(ref_dy)) <= TOL
+    assert (got_rows == ref_dy).mean() >= 0.999
+    assert (dy[ot["slot_src"] < 0] == POISON).all()
+    assert rel_err(dg.reshape(R * S, K), ref_dg) <= TOL
+
+
+def _reduce(cfg, arena, rep_np, home_np, P):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    rep = to_dev(rep_np)
+    home = to_dev(home_np)
+    status = torch.zeros(1, dtype=torch.int32, device=home.device)
+    me.moonep_reduce_grad(cfg, arena, rep, home, P, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return to_np(home)
+
+
+@pytest.mark.parametrize("shape", [(8, 32, 4, 256, 4, 2048), (4, 16, 2, 40, 3, 13),
+                                   (8, 64, 8, 64, 8, 1000), (2, 8, 2, 30, 1, 8)])
+def test_reduce_grad_matches_oracle(shape):
+    R, E, K, S, B, P = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=6.0, seed=6, budget=B)
+    assert int(ot["n_piece"][0]) > 0
+    rep = normal_bf16((R, B, P), seed=6, stream=11)
+    home = normal_bf16((E, P), seed=6, stream=12)
+    got = _reduce(cfg, arena, rep, home, P)
+    ref = oracle.reduce_grad(ocfg, ot, rep, home)
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999
+
+
+def test_reduce_grad_gradient_equivalence_exact():
+    """Integer-valued gradients: home + replicas == the no-replication gradient, bit for bit."""
+    R, E, K, S, B = 8, 32, 4, 64, 4
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=6.0, seed=8, budget=B)
+    P = 24
+    NvS = int(ot["nvs"][0])
+    g = np.random.default_rng(8).integers(-1, 2, size=(R * NvS, P))
+    flat = make_routing(R, E, K, S, 6.0, seed=8)[0].ravel()
+    ref = np.zeros((E, P), np.int64)
+    np.add.at(ref, flat, g[ot["slot_of"]])
+    home = np.zeros((E, P), np.int64)
+    rep = np.zeros((R, B, P), np.int64)
+    L = E // R
+    for d in range(R):
+        for i in range(int(ot["n_seg"][d])):
+            e, s0, ln = ot["seg_expert"][d, i], ot["seg_start"][d, i], ot["seg_len"][d, i]
+            part = g[d * NvS + s0: d * NvS + s0 + ln].sum(0)
+            if i < L:
+                home[e] += part
+            else:
+                rep[d, ot["seg_wslot"][d, i]] += part
+    from moonep_inputs import f32_to_bf16_bits
+    got = _reduce(cfg, arena, f32_to_bf16_bits(rep.astype(np.float32)),
+                  f32_to_bf16_bits(home.astype(np.float32)), P)
+    assert np.array_equal(bf16_bits_to_f32(got).astype(np.int64), ref)
+
+
+def test_reduce_grad_without_budget_is_a_no_op():
+    cfg, ocfg, ot, arena = _setup(4, 16, 2, 40, 8, mv=4.0, seed=9, budget=0, mode=1)
+    home = integer_bf16((16, 16), seed=9)
+    got = _reduce(cfg, arena, np.zeros((4, 0, 16), np.uint16), home, 16)
+    assert np.array_equal(got, home)

@@ -1,0 +1,520 @@
+// Data-movement kernels of the MoonEP hot path: zero-copy dispatch, combine,
+// combine-backward and reduce_grad.  All are HBM-bound row moves with O(1)
+// arithmetic per byte; tensor cores are not involved.
+//
+// Rows are moved as 16-byte vectors (8 bf16).  One warp owns one token: lane k
+// (< K) holds the token's k-th slot and gate and broadcasts them with shuffles.
+// Rows whose byte length or base address is not 16-byte aligned take a scalar
+// (one bf16 per lane) path.
+#include <cuda_bf16.h>
+
+#include "moonep_internal.cuh"
+
+namespace moonep {
+
+namespace {
+
+constexpr int kWarpsPerBlock = 8;
+constexpr int kThreads = kWarpsPerBlock * 32;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat16 l = __float2bfloat16_rn(lo);
+  const __nv_bfloat16 h = __float2bfloat16_rn(hi);
+  return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
+}
+
+__device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f_to_bf16(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// slot of pair (t, lane) for lanes < K, validated against the buffer; -1 otherwise
+__device__ __forceinline__ int load_slot(const int32_t *slot_of, int64_t t, int K, int64_t nrows,
+                                         int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  int s = -1;
+  if (lane < K) {
+    s = __ldg(slot_of + t * K + lane);
+    if (s >= nrows || s < -1) {
+      set_status(status, MOONEP_DEV_BAD_PLAN);
+      s = -1;
+    }
+  }
+  return s;
+}
+
+// ------------------------------------------------------------- dispatch ---
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+dispatch_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ x,
+                    uint4 *__restrict__ recv, int64_t T, int K, int64_t nvec, int64_t nrows,
+                    int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const uint4 *src = x + t * nvec;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      uint4 buf[U];
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) buf[u] = __ldcs(src + v);
+      }
+      for (int k = 0; k < K; k++) {
+        const int row = __shfl_sync(0xffffffffu, my_slot, k);
+        if (row < 0) continue;
+        uint4 *dst = recv + (int64_t)row * nvec;
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          if (v < nvec) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+dispatch_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ x,
+                       uint16_t *__restrict__ recv, int64_t T, int K, int64_t H, int64_t nrows,
+                       int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    for (int64_t h0 = 0; h0 < H; h0 += 32) {
+      const int64_t h = h0 + lane;
+      const uint16_t v = h < H ? x[t * H + h] : 0;
+      for (int k = 0; k < K; k++) {
+        const int row = __shfl_sync(0xffffffffu, my_slot, k);
+        if (row >= 0 && h < H) recv[(int64_t)row * H + h] = v;
+      }
+    }
+  }
+}
+
+// -------------------------------------------------------------- combine ---
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+combine_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ y,
+                   const float *__restrict__ gates, uint4 *__restrict__ out, int64_t T, int K,
+                   int64_t nvec, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      float acc[U][8];
+#pragma unroll
+      for (int u = 0; u < U; u++)
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[u][i] = 0.f;
+      for (int k = 0; k < K; k++) {
+        const int row = __shfl_sync(0xffffffffu, my_slot, k);
+        const float w = __shfl_sync(0xffffffffu, my_w, k);
+        if (row < 0) continue;
+        const uint4 *src = y + (int64_t)row * nvec;
+        uint4 q[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          if (v < nvec) q[u] = __ldcs(src + v);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const uint32_t wd[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            acc[u][2 * i] = __fmaf_rn(w, bf16_lo(wd[i]), acc[u][2 * i]);
+            acc[u][2 * i + 1] = __fmaf_rn(w, bf16_hi(wd[i]), acc[u][2 * i + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+          o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+          o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+          o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+          out[t * nvec + v] = o;
+        }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+combine_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ y,
+                      const float *__restrict__ gates, uint16_t *__restrict__ out, int64_t T, int K,
+                      int64_t H, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? gates[t * K + lane] : 0.f;
+    for (int64_t h0 = 0; h0 < H; h0 += 32) {
+      const int64_t h = h0 + lane;
+      float acc = 0.f;
+      for (int k = 0; k < K; k++) {
+        const int row = __shfl_sync(0xffffffffu, my_slot, k);
+        const float w = __shfl_sync(0xffffffffu, my_w, k);
+        if (row >= 0 && h < H) acc = __fmaf_rn(w, bf16_to_f(y[(int64_t)row * H + h]), acc);
+      }
+      if (h < H) out[t * H + h] = f_to_bf16(acc);
+    }
+  }
+}
+
+// ----------------------------------------------------- combine-backward ---
+// dy[slot_k] = bf16(w_k * dout[t]); dgates[t,k] = <dout[t], y[slot_k]> (fp32, lane
+// partials then a warp tree).  One k at a time; the dout row is re-read from
+// cache for each k.
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+combine_bwd_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ dout,
+                       const uint4 *__restrict__ y, const float *__restrict__ gates,
+                       uint4 *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
+                       int64_t nvec, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    const uint4 *g = dout + t * nvec;
+    float my_dg = 0.f;
+    for (int k = 0; k < K; k++) {
+      const int row = __shfl_sync(0xffffffffu, my_slot, k);
+      const float w = __shfl_sync(0xffffffffu, my_w, k);
+      float part = 0.f;
+      if (row >= 0) {
+        const uint4 *yr = y + (int64_t)row * nvec;
+        uint4 *dr = dy + (int64_t)row * nvec;
+        for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+          uint4 gq[U], yq[U];
+#pragma unroll
+          for (int u = 0; u < U; u++) {
+            const int64_t v = v0 + u * 32 + lane;
+            if (v < nvec) {
+              gq[u] = __ldg(g + v);
+              yq[u] = __ldcs(yr + v);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < U; u++) {
+            const int64_t v = v0 + u * 32 + lane;
+            if (v < nvec) {
+              const uint32_t gw[4] = {gq[u].x, gq[u].y, gq[u].z, gq[u].w};
+              const uint32_t yw[4] = {yq[u].x, yq[u].y, yq[u].z, yq[u].w};
+              uint32_t o[4];
+#pragma unroll
+              for (int i = 0; i < 4; i++) {
+                const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+                part = __fmaf_rn(g0, bf16_lo(yw[i]), part);
+                part = __fmaf_rn(g1, bf16_hi(yw[i]), part);
+                o[i] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+              }
+              dr[v] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (lane == k) my_dg = part;
+    }
+    if (lane < K) dgates[t * K + lane] = my_dg;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ dout,
+                          const uint16_t *__restrict__ y, const float *__restrict__ gates,
+                          uint16_t *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
+                          int64_t H, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? gates[t * K + lane] : 0.f;
+    float my_dg = 0.f;
+    for (int k = 0; k < K; k++) {
+      const int row = __shfl_sync(0xffffffffu, my_slot, k);
+      const float w = __shfl_sync(0xffffffffu, my_w, k);
+      float part = 0.f;
+      if (row >= 0) {
+        for (int64_t h = lane; h < H; h += 32) {
+          const float g = bf16_to_f(dout[t * H + h]);
+          part = __fmaf_rn(g, bf16_to_f(y[(int64_t)row * H + h]), part);
+          dy[(int64_t)row * H + h] = f_to_bf16(__fmul_rn(w, g));
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (lane == k) my_dg = part;
+    }
+    if (lane < K) dgates[t * K + lane] = my_dg;
+  }
+}
+
+// ----------------------------------------------------------- reduce_grad ---
+// Work units: (replicated expert, column vector).  Each unit reads the home
+// vector, adds the expert's local replica vectors in plan order, writes home.
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
+                       const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
+                       const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
+                       const uint4 *__restrict__ rep, uint4 *__restrict__ home, int64_t nvec,
+                       int R, int E, int B, int PMAX, int32_t *status) {
+  int64_t n_exp = scalars[S_N_REPLICATED];
+  if (n_exp < 0 || n_exp > E) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+    n_exp = 0;
+  }
+  const int64_t per_exp = (nvec + 32 * U - 1) / (32 * U);  // warp-chunks per expert
+  const int64_t total = n_exp * per_exp;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t w = warp_g; w < total; w += nwarps) {
+    const int e = replicated[w / per_exp];
+    const int64_t v0 = (w % per_exp) * 32 * U;
+    const int b = e >= 0 && e < E ? pbeg[e] : 0, en = e >= 0 && e < E ? pend[e] : -1;
+    if (e < 0 || e >= E || b < 0 || en > PMAX || en < b) {
+      if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+      continue;
+    }
+    float acc[U][8];
+    uint4 *hrow = home + (int64_t)e * nvec;
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + u * 32 + lane;
+      uint4 q = make_uint4(0, 0, 0, 0);
+      if (v < nvec) q = hrow[v];
+      const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        acc[u][2 * i] = bf16_lo(wd[i]);
+        acc[u][2 * i + 1] = bf16_hi(wd[i]);
+      }
+    }
+    for (int pc = b; pc < en; pc++) {
+      const int ws = pwslot[pc], rk = prank[pc];
+      if (ws < 0) continue;
+      if (ws >= B || rk < 0 || rk >= R) {
+        if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+        continue;
+      }
+      const uint4 *rrow = rep + ((int64_t)rk * B + ws) * nvec;
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) {
+          const uint4 q = __ldcs(rrow + v);
+          const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            acc[u][2 * i] = __fadd_rn(acc[u][2 * i], bf16_lo(wd[i]));
+            acc[u][2 * i + 1] = __fadd_rn(acc[u][2 * i + 1], bf16_hi(wd[i]));
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + u * 32 + lane;
+      if (v < nvec) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        hrow[v] = o;
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
+                          const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
+                          const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
+                          const uint16_t *__restrict__ rep, uint16_t *__restrict__ home, int64_t P,
+                          int R, int E, int B, int PMAX, int32_t *status) {
+  int64_t n_exp = scalars[S_N_REPLICATED];
+  if (n_exp < 0 || n_exp > E) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+    n_exp = 0;
+  }
+  const int64_t total = n_exp * P;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {
+    const int e = replicated[q / P];
+    const int64_t c = q % P;
+    const int b = e >= 0 && e < E ? pbeg[e] : 0, en = e >= 0 && e < E ? pend[e] : -1;
+    if (e < 0 || e >= E || b < 0 || en > PMAX || en < b) {
+      set_status(status, MOONEP_DEV_BAD_PLAN);
+      continue;
+    }
+    float acc = bf16_to_f(home[(int64_t)e * P + c]);
+    for (int pc = b; pc < en; pc++) {
+      const int ws = pwslot[pc], rk = prank[pc];
+      if (ws < 0) continue;
+      if (ws >= B || rk < 0 || rk >= R) {
+        set_status(status, MOONEP_DEV_BAD_PLAN);
+        continue;
+      }
+      acc = __fadd_rn(acc, bf16_to_f(rep[((int64_t)rk * B + ws) * P + c]));
+    }
+    home[(int64_t)e * P + c] = f_to_bf16(acc);
+  }
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  return sms;
+}
+
+unsigned token_grid(int64_t T) {
+  int64_t blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int64_t cap = (int64_t)num_sms() * 64;
+  if (blocks > cap) blocks = cap;
+  return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+
+bool data_dims(const moonep_config_t *cfg, Dims *d) {
+  return make_dims(cfg, d) && d->H >= 1;
+}
+
+}  // namespace
+
+}  // namespace moonep
+
+using namespace moonep;
+
+extern "C" moonep_status_t moonep_dispatch(const moonep_config_t *cfg, const void *plan_arena,
+                                           const uint16_t *x, uint16_t *recv, int32_t *dev_status,
+                                           moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!x || !recv || !aligned256(plan_arena)) return MOONEP_ERR_INVALID_ARG;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS;
+  if (d.H % 8 == 0 && aligned16(x) && aligned16(recv)) {
+    dispatch_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(recv), T,
+        (int)d.K, d.H / 8, nrows, dev_status);
+  } else {
+    dispatch_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], x, recv, T, (int)d.K,
+                                                               d.H, nrows, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_combine(const moonep_config_t *cfg, const void *plan_arena,
+                                          const uint16_t *y, const float *gates, uint16_t *out,
+                                          int32_t *dev_status, moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!y || !gates || !out || !aligned256(plan_arena)) return MOONEP_ERR_INVALID_ARG;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS;
+  if (d.H % 8 == 0 && aligned16(y) && aligned16(out)) {
+    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
+        T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else {
+    combine_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], y, gates, out, T,
+                                                              (int)d.K, d.H, nrows, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_combine_backward(const moonep_config_t *cfg,
+                                                   const void *plan_arena, const uint16_t *dout,
+                                                   const uint16_t *y, const float *gates,
+                                                   uint16_t *dy, float *dgates,
+                                                   int32_t *dev_status, moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!dout || !y || !gates || !dy || !dgates || !aligned256(plan_arena))
+    return MOONEP_ERR_INVALID_ARG;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS;
+  if (d.H % 8 == 0 && aligned16(dout) && aligned16(y) && aligned16(dy)) {
+    combine_bwd_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(dout), reinterpret_cast<const uint4 *>(y),
+        gates, reinterpret_cast<uint4 *>(dy), dgates, T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else {
+    combine_bwd_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], dout, y, gates, dy, dgates, T, (int)d.K, d.H, nrows, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
+                                              const uint16_t *rep_grads, uint16_t *home_grads,
+                                              int64_t P_elems, int32_t *dev_status,
+                                              moonep_stream_t stream) {
+  Dims d;
+  if (!make_dims(cfg, &d) || !plan_arena || !dev_status || P_elems < 1)
+    return MOONEP_ERR_INVALID_ARG;
+  if (!home_grads || (d.B > 0 && !rep_grads) || !aligned256(plan_arena))
+    return MOONEP_ERR_INVALID_ARG;
+  if (d.B == 0) return MOONEP_OK;  // no replica slots, nothing to fold
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const unsigned grid = (unsigned)num_sms() * 8;
+  if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
+    reduce_grad_vec_kernel<4><<<grid, kThreads, 0, st>>>(
+        P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
+        P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(rep_grads),
+        reinterpret_cast<uint4 *>(home_grads), P_elems / 8, (int)d.R, (int)d.E, (int)d.B,
+        (int)d.PMAX, dev_status);
+  } else {
+    reduce_grad_scalar_kernel<<<grid, kThreads, 0, st>>>(
+        P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
+        P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], rep_grads, home_grads, P_elems, (int)d.R,
+        (int)d.E, (int)d.B, (int)d.PMAX, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" const char *moonep_status_string(moonep_status_t s) {
+  switch (s) {
+    case MOONEP_OK: return "ok";
+    case MOONEP_ERR_INVALID_ARG: return "invalid argument (config out of range, null or misaligned pointer)";
+    case MOONEP_ERR_CUDA: return "CUDA launch or runtime error";
+    case MOONEP_ERR_UNSUPPORTED: return "sizes past the supported limits";
+  }
+  return "unknown status";
+}

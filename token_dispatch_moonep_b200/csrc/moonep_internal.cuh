@@ -1,0 +1,145 @@
+// Internal definitions shared by the libmoonep.so translation units: arena and
+// workspace layout, config validation, device helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moonep.h"
+
+namespace moonep {
+
+constexpr int kPlanThreads = 512;         // threads of the histogram / solve kernel
+constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kPairsPerThread = 16;        // pairs per thread in the histogram pass
+constexpr int kChunk = kPlanThreads * kPairsPerThread;  // pairs per histogram chunk (8192)
+constexpr int kPlaceThreads = 256;
+constexpr int kPlacePairsPerThread = 4;
+constexpr int kPlacePairsPerBlock = kPlaceThreads * kPlacePairsPerThread;
+constexpr size_t kAlignBytes = 256;
+
+// ----------------------------------------------------------------- config ---
+struct Dims {
+  int64_t R, E, K, S, H, B, A, L, SK, N, NvS, NC, PMAX;
+  int mode;
+};
+
+__host__ __device__ inline int64_t nvs_of(int64_t S, int64_t K, int64_t E, int64_t A) {
+  int64_t sk = S * K;
+  return sk + (A - 1) * (sk < E ? sk : E);
+}
+
+// Validates everything that does not depend on H; returns false on a bad config.
+inline bool make_dims(const moonep_config_t *c, Dims *d) {
+  if (!c) return false;
+  if (c->R < 1 || c->E < 1 || c->E % c->R != 0) return false;
+  if (c->E > MOONEP_MAX_EXPERTS) return false;
+  if (c->K < 1 || c->K > c->E || c->K > MOONEP_MAX_TOPK) return false;
+  if (c->S < 0 || c->budget < 0 || c->budget > c->E) return false;
+  if (c->mode != MOONEP_MODE_TRAIN && c->mode != MOONEP_MODE_INFER) return false;
+  if (c->align < 1 || c->align > 4096) return false;
+  d->R = c->R; d->E = c->E; d->K = c->K; d->S = c->S; d->H = c->H;
+  d->B = c->budget; d->A = c->align; d->mode = c->mode;
+  d->L = d->E / d->R;
+  d->SK = d->S * d->K;
+  d->N = d->R * d->SK;
+  d->NvS = nvs_of(d->S, d->K, d->E, d->A);
+  if (d->N >= (int64_t(1) << 31) || d->R * d->NvS >= (int64_t(1) << 31)) return false;
+  d->NC = d->N > 0 ? (d->N + kChunk - 1) / kChunk : 1;
+  d->PMAX = d->E + d->R;
+  return true;
+}
+
+// ------------------------------------------------------------ plan arena ---
+enum ArenaField {
+  F_SLOT_OF, F_SLOT_SRC, F_EXPERT_COUNT, F_RANK_LOAD, F_OVERFLOW, F_DEFICIT, F_N_SEG,
+  F_SEG_EXPERT, F_SEG_START, F_SEG_LEN, F_SEG_KIND, F_SEG_WSLOT,
+  F_PIECE_EXPERT, F_PIECE_RANK, F_PIECE_START, F_PIECE_LEN, F_PIECE_WSLOT, F_PIECE_OSTART,
+  F_EXP_PIECE_BEGIN, F_EXP_PIECE_END, F_REP_EXPERT, F_REPLICATED, F_SCALARS,
+  F_COUNT
+};
+
+enum Scalar { S_N_PIECE = 0, S_N_REMOTE = 1, S_N_LOCAL = 2, S_N_REPLICATED = 3, S_BAD = 4 };
+
+inline size_t align_up(size_t v) { return (v + kAlignBytes - 1) / kAlignBytes * kAlignBytes; }
+
+struct ArenaLayout {
+  size_t off[F_COUNT];
+  size_t total;
+  explicit ArenaLayout(const Dims &d) {
+    const int64_t n[F_COUNT] = {
+        d.N, d.R * d.NvS, d.E, d.R, d.R, d.R, d.R,
+        d.R * d.E, d.R * d.E, d.R * d.E, d.R * d.E, d.R * d.E,
+        d.PMAX, d.PMAX, d.PMAX, d.PMAX, d.PMAX, d.PMAX,
+        d.E, d.E, d.R * d.B, d.E, 8};
+    size_t o = 0;
+    for (int i = 0; i < F_COUNT; i++) {
+      off[i] = o;
+      o += align_up(size_t(n[i] > 0 ? n[i] : 1) * sizeof(int32_t));
+    }
+    total = o;
+  }
+};
+
+// Device-side bundle of arena pointers.
+struct PlanPtrs {
+  int32_t *f[F_COUNT];
+};
+
+inline PlanPtrs plan_ptrs(const Dims &d, const void *arena) {
+  ArenaLayout lay(d);
+  PlanPtrs p;
+  for (int i = 0; i < F_COUNT; i++)
+    p.f[i] = reinterpret_cast<int32_t *>(const_cast<char *>(static_cast<const char *>(arena)) + lay.off[i]);
+  return p;
+}
+
+// -------------------------------------------------------------- workspace ---
+enum WsField { W_COUNTER, W_HIST, W_RANK, W_EXP_KEPT, W_EXP_ROW0, W_EXP_OSTART, W_PIECE_GROW, W_COUNT };
+
+struct WsLayout {
+  size_t off[W_COUNT];
+  size_t total;
+  explicit WsLayout(const Dims &d) {
+    const size_t n[W_COUNT] = {
+        8 * sizeof(int32_t),
+        size_t(d.E * d.NC) * sizeof(int32_t),
+        size_t(d.N > 0 ? d.N : 1) * sizeof(uint16_t),
+        size_t(d.E) * sizeof(int32_t), size_t(d.E) * sizeof(int32_t), size_t(d.E) * sizeof(int32_t),
+        size_t(d.PMAX) * sizeof(int32_t)};
+    size_t o = 0;
+    for (int i = 0; i < W_COUNT; i++) {
+      off[i] = o;
+      o += align_up(n[i]);
+    }
+    total = o;
+  }
+};
+
+// ---------------------------------------------------------------- helpers ---
+__device__ __forceinline__ void set_status(int32_t *st, int32_t bits) {
+  if (st) atomicOr(st, bits);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+inline cudaStream_t to_cuda(moonep_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace moonep
