@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the MoonEP balanced expert-parallel hot path on B200.
+
+One step = one MoE layer's pass of the whole hot path over a fresh batch of
+router output: plan -> zero-copy dispatch -> identity expert -> combine, and in
+training mode combine-backward -> reduce_grad of replica expert gradients.
+Inputs are synthetic and seeded (Zipf-popular experts, Gumbel-top-k picks,
+softmax gates, N(0,1) bf16 rows; see moonep_inputs).
+
+Metric (headline): dispatch+combine HBM GB/s = algorithmic bytes of the two
+kernels / their CUDA-event time inside the timed steps, plus plan µs per layer.
+Default workload: R=8 ranks, E=256 experts, K=8, S=4096 tokens/rank, H=7168,
+maxvio 0.2, replica budget 32 (training).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--maxvio M]
+    python bench.py --sweep            # maxvio 0.2..20 x 5 seeds, one JSON line per maxvio
+    python bench.py --impl reference   # the CPU oracle on a bounded sample, same metric
+
+With N > 1 (torchrun), every rank runs an independent replica of the layer on
+its own GPU (weak scaling, no data-path collective); rank 0 prints one line
+with the whole-job value (bytes of all ranks / the slowest rank's time).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from moonep_inputs import (MODE_TRAIN, WORKLOADS, make_dout, make_gates, make_routing,  # noqa: E402
+                           make_x)
+
+METRIC = "dispatch+combine HBM GB/s (% of peak) and plan µs/layer vs maxvio, 1×B200"
+DEFAULT_WORKLOAD = "ep8_e256_k8_s4096_h7168"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+# ------------------------------------------------------------------ bytes ---
+def algorithmic_bytes(R, S, K, H, n_local=0, n_rep_exp=0, P=0):
+    """Bytes each kernel must move (bf16 = 2 B), per launch; re-reads and padding excluded."""
+    T = R * S
+    RSK = T * K
+    return {
+        "plan": RSK * 4 * 2,  # router ids in, slot map out
+        "dispatch": T * H * 2 + RSK * H * 2 + RSK * 4,
+        "combine": RSK * H * 2 + T * H * 2 + RSK * 8,
+        "combine_bwd": T * H * 2 + 2 * RSK * H * 2 + RSK * 12,
+        "reduce_grad": n_local * P * 2 + n_rep_exp * P * 2 * 2,
+    }
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic():
+    """Per-kernel DRAM bytes per launch from the committed ncu summary, if still current."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    out = {}
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return out
+    src_hash = {}
+    for f in ("plan.cu", "data.cu", "moonep_internal.cuh"):
+        try:
+            with open(os.path.join(ROOT, "token_dispatch_moonep_b200", "csrc", f), "rb") as fh:
+                src_hash[f] = hashlib.sha256(fh.read()).hexdigest()[:16]
+        except OSError:
+            pass
+    for ln in lines:
+        if ln.startswith("#") or not ln.strip():
+            continue
+        parts = dict(kv.split("=", 1) for kv in ln.split())
+        if src_hash.get(parts.get("source")) == parts.get("sha"):
+            out[parts["kernel"]] = float(parts["bytes_per_launch"])
+    return out
+
+
+# ----------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        import torch
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------- GPU layer ---
+class Layer:
+    """Device buffers and the per-step call sequence of one MoE layer."""
+
+    def __init__(self, w, maxvio, seed, device, with_backward=None, host_inputs=True):
+        import torch
+        import token_dispatch_moonep_b200 as me
+        self.me, self.torch, self.w = me, torch, w
+        self.dev = device
+        self.train = (w.mode == MODE_TRAIN) if with_backward is None else with_backward
+        R, E, K, S, H = w.R, w.E, w.K, w.S, w.H
+        self.cfg = me.Config.of(w)
+        self.NvS = me.moonep_nvs(self.cfg)
+        T = R * S
+        idx, self.alpha, self.maxvio = make_routing(R, E, K, S, maxvio, seed)
+        gates = make_gates(R, S, K, seed)
+        # pinned host copies (for the end-to-end measurement) and device copies
+        pin = torch.cuda.is_available()
+        self.h_idx = torch.from_numpy(idx.ravel().copy())
+        self.h_gates = torch.from_numpy(gates.ravel().copy())
+        if host_inputs:
+            self.h_x = torch.from_numpy(make_x(R, S, H, seed).reshape(-1).view(np.int16))
+            self.h_dout = (torch.from_numpy(make_dout(R, S, H, seed).reshape(-1).view(np.int16))
+                           if self.train else None)
+        else:
+            g = torch.Generator(device=device).manual_seed(seed)
+            self.h_x = torch.randn(T * H, generator=g, device=device).to(torch.bfloat16).view(torch.int16).cpu()
+            self.h_dout = (torch.randn(T * H, generator=g, device=device).to(torch.bfloat16)
+                           .view(torch.int16).cpu() if self.train else None)
+        if pin:
+            self.h_idx = self.h_idx.pin_memory()
+            self.h_gates = self.h_gates.pin_memory()
+            self.h_x = self.h_x.pin_memory()
+            if self.h_dout is not None:
+                self.h_dout = self.h_dout.pin_memory()
+        self.idx = self.h_idx.to(device)
+        self.gates = self.h_gates.to(device)
+        self.x = self.h_x.to(device)
+        self.recv = torch.empty(R * self.NvS * H, dtype=torch.int16, device=device)
+        self.out = torch.empty(T * H, dtype=torch.int16, device=device)
+        self.arena, self.ws, self.status = me.alloc_plan(self.cfg, device)
+        if self.train:
+            self.P = w.P or 2048 * H
+            self.dout = self.h_dout.to(device)
+            self.dy = torch.empty_like(self.recv)
+            self.dg = torch.empty(T * K, dtype=torch.float32, device=device)
+            g = torch.Generator(device=device).manual_seed(seed + 1)
+            self.rep = torch.empty(R * w.budget * self.P, dtype=torch.bfloat16, device=device)
+            self.home = torch.empty(E * self.P, dtype=torch.bfloat16, device=device)
+            for buf in (self.rep, self.home):  # N(0,1) in chunks to bound fp32 temporaries
+                n = buf.numel()
+                step = 1 << 28
+                for i in range(0, n, step):
+                    buf[i:i + step].copy_(torch.randn(min(step, n - i), generator=g, device=device))
+            self.h_out = torch.empty(T * H, dtype=torch.int16).pin_memory() if pin else None
+            self.h_dg = torch.empty(T * K, dtype=torch.float32).pin_memory() if pin else None
+        else:
+            self.P = 0
+            self.h_out = torch.empty(T * H, dtype=torch.int16).pin_memory() if pin else None
+        self.launches_per_step = 4 + (2 if self.train else 0)  # plan = 2 kernels (+1 memset)
+        self.n_local = self.n_rep_exp = 0
+
+    def ops(self):
+        me, c = self.me, self.cfg
+        seq = [("plan", lambda: me.moonep_plan(c, self.idx, self.arena, self.ws, self.status)),
+               ("dispatch", lambda: me.moonep_dispatch(c, self.arena, self.x, self.recv, self.status)),
+               ("combine", lambda: me.moonep_combine(c, self.arena, self.recv, self.gates, self.out,
+                                                     self.status))]
+        if self.train:
+            seq += [("combine_bwd", lambda: me.moonep_combine_backward(
+                        c, self.arena, self.dout, self.recv, self.gates, self.dy, self.dg,
+                        self.status)),
+                    ("reduce_grad", lambda: me.moonep_reduce_grad(c, self.arena, self.rep, self.home,
+                                                                  self.P, self.status))]
+        return seq
+
+    def read_plan_stats(self):
+        v = self.me.moonep_plan_view(self.cfg, self.arena)
+        sc = v["scalars"].cpu().numpy()
+        self.n_local, self.n_rep_exp = int(sc[2]), int(sc[3])
+        self.n_piece, self.n_remote = int(sc[0]), int(sc[1])
+
+    def bytes(self):
+        w = self.w
+        b = algorithmic_bytes(w.R, w.S, w.K, w.H, self.n_local, self.n_rep_exp, self.P)
+        if not self.train:
+            b.pop("combine_bwd")
+            b.pop("reduce_grad")
+        return b
+
+
+def time_steps(layer, steps, warmup, barrier=None):
+    """Warm up, then time `steps` steps with per-kernel CUDA events on the current stream."""
+    torch = layer.torch
+    ops = layer.ops()
+    for _ in range(warmup):
+        for _, fn in ops:
+            fn()
+    torch.cuda.synchronize()
+    layer.read_plan_stats()
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(steps)]
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    time.sleep(0.25)  # let the sampler start before the timed region
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        ev[s][0].record(stream)
+        for i, (_, fn) in enumerate(ops):
+            fn()
+            ev[s][i + 1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if barrier:
+        barrier()
+    total_ms = t0.elapsed_time(t1)
+    per = {name: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)]
+           for i, (name, _) in enumerate(ops)}
+    st = int(layer.status.item())
+    return total_ms, per, clocks, st
+
+
+def time_e2e(layer, steps):
+    """Same step through the public API with host inputs: pinned H2D in, D2H of the results."""
+    torch = layer.torch
+    ops = layer.ops()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        layer.idx.copy_(layer.h_idx, non_blocking=True)
+        layer.gates.copy_(layer.h_gates, non_blocking=True)
+        layer.x.copy_(layer.h_x, non_blocking=True)
+        if layer.train:
+            layer.dout.copy_(layer.h_dout, non_blocking=True)
+        for _, fn in ops:
+            fn()
+        layer.h_out.copy_(layer.out, non_blocking=True)
+        if layer.train:
+            layer.h_dg.copy_(layer.dg, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    h2d = (layer.h_idx.numel() * 4 + layer.h_gates.numel() * 4 + layer.h_x.numel() * 2 +
+           (layer.h_dout.numel() * 2 if layer.train else 0))
+    d2h = layer.h_out.numel() * 2 + (layer.h_dg.numel() * 4 if layer.train else 0)
+    return ms, h2d, d2h
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def oracle_sample_run(w, maxvio, seed, s_sample, budget_s=10.0, min_reps=1):
+    """Time the CPU oracle (plan + dispatch + combine) on the first `s_sample` tokens of
+    every rank of the workload's routing, repeated until `budget_s` seconds pass."""
+    import oracle
+    R, E, K, H = w.R, w.E, w.K, w.H
+    idx, _, _ = make_routing(R, E, K, w.S, maxvio, seed)
+    idx = np.ascontiguousarray(idx[:, :s_sample, :])
+    gates = np.ascontiguousarray(make_gates(R, w.S, K, seed)[:, :s_sample, :])
+    x = make_x(R, s_sample, H, seed).reshape(R * s_sample, H)
+    cfg = oracle.Config(R=R, E=E, K=K, S=s_sample, H=H, budget=w.budget, mode=w.mode)
+    b = algorithmic_bytes(R, s_sample, K, H)
+    reps, t_plan, t_dc = 0, 0.0, 0.0
+    t_start = time.perf_counter()
+    while reps < min_reps or time.perf_counter() - t_start < budget_s:
+        a = time.perf_counter()
+        st, t = oracle.plan(cfg, idx)
+        m = time.perf_counter()
+        recv = oracle.dispatch(cfg, t["slot_of"], x)
+        oracle.combine(cfg, t["slot_of"], recv, gates)
+        e = time.perf_counter()
+        t_plan += m - a
+        t_dc += e - m
+        reps += 1
+    gbs = (b["dispatch"] + b["combine"]) * reps / t_dc / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "plan_us": t_plan / reps * 1e6, "reps": reps, "seconds": t_dc + t_plan,
+            "sample": f"first {s_sample} of {w.S} tokens on each of the {R} ranks of the "
+                      f"same seeded routing (maxvio {maxvio}), planned as one layer; "
+                      f"plan + dispatch + combine, single-threaded C, repeated {reps}x"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, on the same metric, on a bounded sample per step."""
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    mv = args.maxvio if args.maxvio is not None else w.maxvio[0]
+    s_sample = max(1, min(w.S, 8 if w.H >= 4096 else 64))
+    import oracle
+    R, E, K, H = w.R, w.E, w.K, w.H
+    idx, _, _ = make_routing(R, E, K, w.S, mv, args.seed)
+    gates = make_gates(R, w.S, K, args.seed)
+    x_full = None
+    b = algorithmic_bytes(R, s_sample, K, H)
+    cfg = oracle.Config(R=R, E=E, K=K, S=s_sample, H=H, budget=w.budget, mode=w.mode)
+    times, plan_t = [], []
+    deadline = time.perf_counter() + args.reference_budget_s
+    done = 0
+    for step in range(args.warmup + args.steps):
+        # step s uses the s-th slice of s_sample tokens of every rank (wrapping)
+        lo = (step * s_sample) % max(1, w.S - s_sample + 1)
+        si = np.ascontiguousarray(idx[:, lo:lo + s_sample, :])
+        sg = np.ascontiguousarray(gates[:, lo:lo + s_sample, :])
+        x = make_x(R, s_sample, H, args.seed + step).reshape(R * s_sample, H)
+        a = time.perf_counter()
+        st, t = oracle.plan(cfg, si)
+        m = time.perf_counter()
+        recv = oracle.dispatch(cfg, t["slot_of"], x)
+        oracle.combine(cfg, t["slot_of"], recv, sg)
+        e = time.perf_counter()
+        if step >= args.warmup:
+            times.append(e - m)
+            plan_t.append(m - a)
+            done += 1
+        if time.perf_counter() > deadline and done >= 1:
+            break
+    gbs = (b["dispatch"] + b["combine"]) * done / sum(times) / 1e9
+    sample = (f"per step {s_sample} tokens on each of the {R} ranks (a slice of the seeded "
+              f"{args.workload} routing, maxvio {mv}), planned as one layer; plan + dispatch + "
+              "combine in the single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": done, "warmup": args.warmup, "ms_per_step": 1e3 * (sum(times) + sum(plan_t)) / done,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": args.workload, "maxvio": mv,
+                                        "sample_tokens_per_rank": s_sample},
+        "plan_us_per_layer": 1e6 * sum(plan_t) / done,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main ---
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--maxvio", type=float, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
+    ap.add_argument("--sweep", action="store_true", help="maxvio sweep of the workload shape")
+    ap.add_argument("--scale-s", type=int, default=1, help="divide S (tokens/rank) by this (profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--reference-budget-s", type=float, default=120.0)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+
+    def barrier():
+        if pg:
+            pg.barrier()
+
+    w = WORKLOADS[args.workload]
+    if args.scale_s > 1:  # a smaller case of the same shape (profiling captures)
+        import dataclasses
+        w = dataclasses.replace(w, S=max(1, w.S // args.scale_s),
+                                P=max(8, (w.P or 2048 * w.H) // args.scale_s))
+    if args.sweep:
+        return run_sweep(args, w, device)
+    mv = args.maxvio if args.maxvio is not None else w.maxvio[0]
+    layer = Layer(w, mv, args.seed + rank, device)
+    total_ms, per, clocks, st = time_steps(layer, args.steps, args.warmup, barrier)
+    b = layer.bytes()
+
+    dc_ms = sum(per["dispatch"]) + sum(per["combine"])
+    if pg:
+        t = torch.tensor([total_ms, dc_ms], dtype=torch.float64, device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, dc_ms = t.tolist()
+    dc_bytes = (b["dispatch"] + b["combine"]) * args.steps * world
+    value = dc_bytes / (dc_ms * 1e-3) / 1e9
+    peak, peak_src = hbm_peak()
+
+    kern = {}
+    for name, ts in per.items():
+        avg = sum(ts) / len(ts)
+        kern[name] = {"ms": avg, "bytes": b[name], "GBs": b[name] / (avg * 1e-3) / 1e9,
+                      "frac": b[name] / (avg * 1e-3) / 1e9 / peak, "share": sum(ts) / total_ms}
+    kern["plan"].pop("frac")
+    dom = max((k for k in kern if k != "plan"), key=lambda k: kern[k]["ms"])
+    traffic = ncu_traffic().get(dom)
+    roof = {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["GBs"], "peak": peak,
+            "unit": "GB/s", "frac": kern[dom]["GBs"] / peak, "traffic": traffic,
+            "peak_source": f"{peak_src} copy bandwidth"}
+
+    e2e = None
+    if not args.no_e2e:
+        ms, h2d, d2h = time_e2e(layer, min(args.steps, 20))
+        n = min(args.steps, 20)
+        e2e = {"value": (b["dispatch"] + b["combine"]) * n * world / (ms * 1e-3) / 1e9,
+               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ms / n, "steps": n}
+        if pg:
+            t = torch.tensor([ms], dtype=torch.float64, device=device)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e["value"] = (b["dispatch"] + b["combine"]) * n * world / (t.item() * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = oracle_sample_run(w, mv, args.seed, s_sample=min(w.S, 64 if w.H >= 4096 else 256))
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name + (f"/S{w.S}" if args.scale_s > 1 else ""),
+                       "R": w.R, "E": w.E, "K": w.K, "S": w.S, "H": w.H, "budget": w.budget,
+                       "mode": "train" if w.mode == MODE_TRAIN else "infer",
+                       "maxvio": round(layer.maxvio, 4), "zipf_alpha": round(layer.alpha, 4),
+                       "step": "plan+dispatch+combine" + ("+combine_bwd+reduce_grad" if layer.train else ""),
+                       "grad_elems_per_expert": layer.P,
+                       "l2": "inputs larger than L2 (x %.0f MB, dispatch buffer %.0f MB); no flush"
+                             % (layer.x.numel() * 2 / 1e6, layer.recv.numel() * 2 / 1e6),
+                       "parallelism": f"{world} independent replica(s), one per GPU"},
+            "pct_of_peak": {"measured": value / peak, "nominal_8TBs": value / NOMINAL_HBM_GBS},
+            "plan_us_per_layer": kern["plan"]["ms"] * 1e3,
+            "layer_us": 1e3 * (kern["plan"]["ms"] + kern["dispatch"]["ms"] + kern["combine"]["ms"]),
+            "kernels": kern,
+            "replicas": {"pieces": layer.n_piece, "local": layer.n_local, "remote": layer.n_remote,
+                         "experts_replicated": layer.n_rep_exp},
+            "device_status": st,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": layer.launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def run_sweep(args, w, device):
+    """Plan µs and dispatch/combine GB/s per maxvio (5 seeds each), plus flatness.
+    Forward only (plan + dispatch + combine), the per-layer time the pages plot."""
+    rows = []
+    peak, _ = hbm_peak()
+    targets = (0.2, 1.0, 2.0, 5.0, 10.0, 20.0) if args.maxvio is None else (args.maxvio,)
+    seeds = (0, 1, 2, 3, 4)
+    for mv in targets:
+        per_seed = []
+        for seed in seeds:
+            layer = Layer(w, mv, seed, device, with_backward=False, host_inputs=False)
+            total_ms, per, clocks, st = time_steps(layer, max(20, args.steps // 10), args.warmup)
+            b = layer.bytes()
+            med = {k: statistics.median(v) for k, v in per.items()}
+            per_seed.append({"seed": seed, "maxvio": layer.maxvio, "alpha": layer.alpha,
+                             "plan_us": med["plan"] * 1e3,
+                             "dispatch_GBs": b["dispatch"] / med["dispatch"] / 1e6,
+                             "combine_GBs": b["combine"] / med["combine"] / 1e6,
+                             "layer_us": 1e3 * (med["plan"] + med["dispatch"] + med["combine"]),
+                             "pieces": layer.n_piece, "status": st, "clocks": clocks})
+            del layer
+            import torch
+            torch.cuda.empty_cache()
+        row = {"target_maxvio": mv,
+               "maxvio": statistics.mean(r["maxvio"] for r in per_seed),
+               "plan_us": statistics.mean(r["plan_us"] for r in per_seed),
+               "dispatch_GBs": statistics.mean(r["dispatch_GBs"] for r in per_seed),
+               "combine_GBs": statistics.mean(r["combine_GBs"] for r in per_seed),
+               "layer_us": statistics.mean(r["layer_us"] for r in per_seed),
+               "pieces": statistics.mean(r["pieces"] for r in per_seed),
+               "seeds": per_seed}
+        rows.append(row)
+        print(json.dumps({k: v for k, v in row.items() if k != "seeds"}), flush=True)
+    lay = [r["layer_us"] for r in rows]
+    print(json.dumps({"sweep": w.name, "flatness_max_over_min_layer_us": max(lay) / min(lay),
+                      "layer_us": lay, "peak_GBs": peak,
+                      "rows": rows}), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
