@@ -146,6 +146,29 @@ MOONEP_API size_t moonep_workspace_bytes(const moonep_config_t *cfg);
 MOONEP_API moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t *topk_idx, void *plan_arena,
                             void *workspace, int32_t *dev_status, moonep_stream_t stream);
 
+/* Allocation-free variant of moonep_plan.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory on their
+ * own — for example a plugin running inside another engine that only hands it
+ * the tensors of one call, or a serving loop that reserved all device memory up
+ * front and must not call cudaMalloc (which can also synchronise the device)
+ * while it runs.  Such a caller passes only inputs and outputs; the plan's
+ * scratch is a fixed array of MOONEP_STATIC_WORKSPACE_BYTES inside the library
+ * (a device global that every GPU which loads the library keeps until exit).
+ *   - Same arguments and results as moonep_plan, without `workspace`.
+ *   - Configs whose moonep_workspace_bytes() exceeds the array are rejected
+ *     with MOONEP_ERR_UNSUPPORTED before anything is enqueued.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.  Nothing is allocated or freed, ever.
+ *   - All calls on a device share the one array: calls whose execution
+ *     overlaps on the GPU (other streams, concurrent graphs) race and must be
+ *     ordered by the caller.  Each call clears what must start at zero. */
+#define MOONEP_STATIC_WORKSPACE_BYTES (4u << 20)
+
+MOONEP_API moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const int32_t *topk_idx,
+                                              void *plan_arena, int32_t *dev_status,
+                                              moonep_stream_t stream);
+
 /* Fill `out` with device pointers into `plan_arena` (pure host arithmetic). */
 MOONEP_API moonep_status_t moonep_plan_view(const moonep_config_t *cfg, const void *plan_arena,
                                  moonep_plan_view_t *out);

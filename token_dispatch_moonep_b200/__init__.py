@@ -9,6 +9,7 @@ The functions keep the C names::
 
     moonep_nvs(cfg) / moonep_plan_bytes(cfg) / moonep_workspace_bytes(cfg)
     moonep_plan(cfg, topk_idx, plan_arena, workspace, dev_status, stream=None)
+    moonep_plan_static(cfg, topk_idx, plan_arena, dev_status, stream=None)
     moonep_plan_view(cfg, plan_arena) -> dict of int32 tensor views
     moonep_dispatch(cfg, plan_arena, x, recv, dev_status, stream=None)
     moonep_combine(cfg, plan_arena, y, gates, out, dev_status, stream=None)
@@ -41,6 +42,7 @@ MODE_TRAIN = 0
 MODE_INFER = 1
 MAX_EXPERTS = 1024
 MAX_TOPK = 32
+STATIC_WORKSPACE_BYTES = 4 << 20
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -110,6 +112,8 @@ _lib.moonep_workspace_bytes.argtypes = [_CP]
 _lib.moonep_workspace_bytes.restype = ctypes.c_size_t
 _lib.moonep_plan.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_plan.restype = _ST
+_lib.moonep_plan_static.argtypes = [_CP, _VP, _VP, _VP, _VP]
+_lib.moonep_plan_static.restype = _ST
 _lib.moonep_plan_view.argtypes = [_CP, _VP, ctypes.POINTER(PlanView)]
 _lib.moonep_plan_view.restype = _ST
 _lib.moonep_dispatch.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
@@ -174,6 +178,14 @@ def moonep_workspace_bytes(cfg: Config) -> int:
 def moonep_plan(cfg: Config, topk_idx, plan_arena, workspace, dev_status, stream=None) -> None:
     _check("moonep_plan", _lib.moonep_plan(ctypes.byref(cfg), _ptr(topk_idx), _ptr(plan_arena),
                                            _ptr(workspace), _ptr(dev_status), _stream(stream)))
+
+
+def moonep_plan_static(cfg: Config, topk_idx, plan_arena, dev_status, stream=None) -> None:
+    """moonep_plan without a caller workspace: the library's fixed scratch array is used
+    (for callers that cannot allocate; see include/moonep.h).  Calls that overlap on the
+    GPU share that array and race."""
+    _check("moonep_plan_static", _lib.moonep_plan_static(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(plan_arena), _ptr(dev_status), _stream(stream)))
 
 
 def moonep_plan_view_ptrs(cfg: Config, plan_arena) -> PlanView:

@@ -15,6 +15,8 @@
 //   plan_place       every pair's final row: position inside its expert's list
 //                    = chunk base + stable rank; the first kept_e positions stay
 //                    in the home segment, the rest map through the piece table.
+#include <atomic>
+
 #include "moonep_internal.cuh"
 
 namespace moonep {
@@ -628,4 +630,36 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
                                                                  kept, row0, ostart, grow);
   if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
   return MOONEP_OK;
+}
+
+// ------------------------------------------------ allocation-free variant ---
+// Scratch for moonep_plan_static: a fixed device array that lives as long as
+// the library is loaded.  Host code cannot use the symbol itself as a device
+// pointer; its device address is looked up once per device.
+static __device__ __align__(256) unsigned char g_plan_scratch[MOONEP_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::atomic<void *> g_plan_scratch_addr[kMaxDevices];
+}  // namespace
+
+extern "C" moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const int32_t *topk_idx,
+                                              void *plan_arena, int32_t *dev_status,
+                                              moonep_stream_t stream) {
+  Dims d;
+  if (!make_dims(cfg, &d)) return MOONEP_ERR_INVALID_ARG;
+  if (WsLayout(d).total > (size_t)MOONEP_STATIC_WORKSPACE_BYTES) return MOONEP_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOONEP_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOONEP_ERR_UNSUPPORTED;
+  void *scratch = g_plan_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
+    if (cudaGetSymbolAddress(&scratch, g_plan_scratch) != cudaSuccess || !scratch)
+      return MOONEP_ERR_CUDA;
+    g_plan_scratch_addr[dev].store(scratch, std::memory_order_release);
+  }
+  // the ordinary plan with the static array as its workspace (it resets the
+  // arrival counter and flags itself; every other scratch word is written
+  // before it is read)
+  return moonep_plan(cfg, topk_idx, plan_arena, scratch, dev_status, stream);
 }
