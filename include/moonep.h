@@ -141,8 +141,9 @@ MOONEP_API size_t moonep_workspace_bytes(const moonep_config_t *cfg);
  *   topk_idx   device int32 [R*S*K] (may be NULL when S == 0)
  *   plan_arena device, moonep_plan_bytes(cfg) bytes, 256-byte aligned; written
  *   workspace  device, moonep_workspace_bytes(cfg) bytes, 256-byte aligned
- *   dev_status device int32, bits OR-ed: BAD_EXPERT_ID, BUDGET, CAPACITY
- * Enqueues one memset and two kernels. */
+ *   dev_status device int32, bits OR-ed: BAD_EXPERT_ID, BUDGET, CAPACITY, TIMEOUT
+ * Enqueues one cooperative kernel (its CTAs are co-resident and wait for each
+ * other with bounded waits, see moonep_debug_set_wait). */
 MOONEP_API moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t *topk_idx, void *plan_arena,
                             void *workspace, int32_t *dev_status, moonep_stream_t stream);
 
@@ -160,14 +161,24 @@ MOONEP_API moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
  *   - The first call on a device (with that device current) looks up the
  *     array's device address once; make that first call before any stream
  *     capture.  Nothing is allocated or freed, ever.
- *   - All calls on a device share the one array: calls whose execution
- *     overlaps on the GPU (other streams, concurrent graphs) race and must be
- *     ordered by the caller.  Each call clears what must start at zero. */
+ *   - All calls on a device share the one array and find it as the previous
+ *     call left it; no word of it needs to start at zero (each is written
+ *     before it is read in the same call, and the arrival flags carry a
+ *     per-launch epoch).  Calls whose execution overlaps on the GPU (other
+ *     streams, concurrent graphs) race and must be ordered by the caller. */
 #define MOONEP_STATIC_WORKSPACE_BYTES (4u << 20)
 
 MOONEP_API moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const int32_t *topk_idx,
                                               void *plan_arena, int32_t *dev_status,
                                               moonep_stream_t stream);
+
+/* Diagnostics for the plan kernel's bounded waits (process-wide, host-side).
+ * The plan is one cooperative launch whose CTAs wait for each other twice;
+ * each wait gives up after `limit_ns` nanoseconds (default 200 ms), sets
+ * MOONEP_DEV_TIMEOUT and leaves an invalid plan (slot_of = -1) instead of
+ * hanging.  `phantom_arrivals` (tests only, 0..32) makes the solving CTA also
+ * wait for that many arrivals that no CTA ever makes, forcing the timeout. */
+MOONEP_API moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals);
 
 /* Fill `out` with device pointers into `plan_arena` (pure host arithmetic). */
 MOONEP_API moonep_status_t moonep_plan_view(const moonep_config_t *cfg, const void *plan_arena,

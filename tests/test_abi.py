@@ -130,3 +130,10 @@ def test_status_strings():
     for s in (me.OK, me.ERR_INVALID_ARG, me.ERR_CUDA, me.ERR_UNSUPPORTED):
         assert me.moonep_status_string(s)
     assert me.moonep_status_string(99) == "unknown status"
+
+
+def test_debug_wait_knob_validates_arguments():
+    assert me._lib.moonep_debug_set_wait(-1, 0) == me.ERR_INVALID_ARG
+    assert me._lib.moonep_debug_set_wait(1000, 33) == me.ERR_INVALID_ARG
+    assert me._lib.moonep_debug_set_wait(1000, -1) == me.ERR_INVALID_ARG
+    assert me._lib.moonep_debug_set_wait(me.DEFAULT_WAIT_NS, 0) == me.OK

@@ -59,6 +59,8 @@ SHAPES = [
     (8, 64, 6, 40, 1, 1),        # H = 1
     (4, 16, 2, 0, 64, 1),        # empty batch
     (8, 64, 8, 1200, 1032, 1),   # several blocks, ragged vector tail (129 vectors per row)
+    (4, 32, 12, 20, 64, 1),      # K > 8: the k-at-a-time kernels
+    (2, 64, 32, 9, 40, 1),       # K = MAX_TOPK
 ]
 
 

@@ -143,3 +143,76 @@ def test_full_size_plans(name, mv, seed):
     ot, gv = _run(w.R, w.E, w.K, w.S, idx, budget=w.budget, mode=w.mode)
     if w.mode == 1 and mv >= 20:
         assert int(ot["n_remote"][0]) > 0  # the remote-read path is exercised
+
+
+def test_several_chunks_per_cta():
+    # 1.28M pairs = 157 chunks of 8192: more chunks than co-resident CTAs
+    idx, _, _ = make_routing(8, 64, 8, 20000, 4.0, seed=9)
+    _run(8, 64, 8, 20000, idx, budget=8)
+
+
+def test_workspace_reuse_with_arbitrary_contents():
+    import torch
+    import token_dispatch_moonep_b200 as me
+    cfg, ocfg = configs(8, 256, 8, 512)
+    arena, ws, _ = me.alloc_plan(cfg)
+    for fill, (mv, seed) in [(0x00, (0.2, 0)), (0xFF, (5.0, 1)), (0xA5, (20.0, 2)), (None, (1.0, 3)),
+                             (None, (1.0, 3))]:
+        if fill is not None:
+            ws.fill_(fill)
+        idx, _, _ = make_routing(8, 256, 8, 512, mv, seed=seed)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        me.moonep_plan(cfg, torch.from_numpy(idx.ravel().copy()).cuda(), arena, ws, st)
+        torch.cuda.synchronize()
+        ost, ot = oracle.plan(ocfg, idx)
+        gv = {k: (v.cpu().numpy() if not isinstance(v, int) else v)
+              for k, v in me.moonep_plan_view(cfg, arena).items()}
+        compare_plans(cfg, ost, ot, int(st.item()), gv)
+
+
+def test_forced_timeout_reports_status_and_context_stays_usable():
+    """A wait that runs out (an arrival nothing makes) ends the kernel with TIMEOUT."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    cfg, ocfg = configs(8, 64, 8, 3000)
+    idx, _, _ = make_routing(8, 64, 8, 3000, 3.0, seed=4)
+    try:
+        me.moonep_debug_set_wait(2_000_000, 1)  # 2 ms, one phantom arrival
+        st, _, gv, _ = gpu_plan(cfg, idx)
+        assert st & me.DEV_TIMEOUT
+        assert (gv["slot_of"] == -1).all() and (gv["slot_src"] == -1).all()
+    finally:
+        me.moonep_debug_set_wait(me.DEFAULT_WAIT_NS, 0)
+    # the context is intact and the next plan is correct
+    ost, ot = oracle.plan(ocfg, idx)
+    st, _, gv, _ = gpu_plan(cfg, idx)
+    compare_plans(cfg, ost, ot, st, gv)
+
+
+def test_plan_replayed_from_a_cuda_graph():
+    """Graph replays reuse the kernel's arguments; the launch epoch must still advance."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S = 8, 256, 8, 1024
+    cfg, ocfg = configs(R, E, K, S)
+    arena, ws, st = me.alloc_plan(cfg)
+    idx_dev = torch.zeros(R * S * K, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        me.moonep_plan(cfg, idx_dev, arena, ws, st, stream=s)  # warm up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        me.moonep_plan(cfg, idx_dev, arena, ws, st, stream=s)
+    for mv, seed in [(0.2, 0), (20.0, 1), (5.0, 2), (5.0, 2)]:
+        idx, _, _ = make_routing(R, E, K, S, mv, seed=seed)
+        idx_dev.copy_(torch.from_numpy(idx.ravel().copy()))
+        st.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ost, ot = oracle.plan(ocfg, idx)
+        gv = {k: (v.cpu().numpy() if not isinstance(v, int) else v)
+              for k, v in me.moonep_plan_view(cfg, arena).items()}
+        compare_plans(cfg, ost, ot, int(st.item()), gv)
+    del g

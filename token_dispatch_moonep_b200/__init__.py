@@ -11,6 +11,7 @@ The functions keep the C names::
     moonep_plan(cfg, topk_idx, plan_arena, workspace, dev_status, stream=None)
     moonep_plan_static(cfg, topk_idx, plan_arena, dev_status, stream=None)
     moonep_plan_view(cfg, plan_arena) -> dict of int32 tensor views
+    moonep_debug_set_wait(limit_ns, phantom_arrivals=0)
     moonep_dispatch(cfg, plan_arena, x, recv, dev_status, stream=None)
     moonep_combine(cfg, plan_arena, y, gates, out, dev_status, stream=None)
     moonep_combine_backward(cfg, plan_arena, dout, y, gates, dy, dgates, dev_status, stream=None)
@@ -114,6 +115,8 @@ _lib.moonep_plan.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_plan.restype = _ST
 _lib.moonep_plan_static.argtypes = [_CP, _VP, _VP, _VP, _VP]
 _lib.moonep_plan_static.restype = _ST
+_lib.moonep_debug_set_wait.argtypes = [ctypes.c_int64, ctypes.c_int32]
+_lib.moonep_debug_set_wait.restype = _ST
 _lib.moonep_plan_view.argtypes = [_CP, _VP, ctypes.POINTER(PlanView)]
 _lib.moonep_plan_view.restype = _ST
 _lib.moonep_dispatch.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
@@ -186,6 +189,14 @@ def moonep_plan_static(cfg: Config, topk_idx, plan_arena, dev_status, stream=Non
     GPU share that array and race."""
     _check("moonep_plan_static", _lib.moonep_plan_static(
         ctypes.byref(cfg), _ptr(topk_idx), _ptr(plan_arena), _ptr(dev_status), _stream(stream)))
+
+
+def moonep_debug_set_wait(limit_ns: int, phantom_arrivals: int = 0) -> None:
+    """Time limit of the plan kernel's in-kernel waits; phantom arrivals force a timeout (tests)."""
+    _check("moonep_debug_set_wait", _lib.moonep_debug_set_wait(int(limit_ns), int(phantom_arrivals)))
+
+
+DEFAULT_WAIT_NS = 200 * 1000 * 1000
 
 
 def moonep_plan_view_ptrs(cfg: Config, plan_arena) -> PlanView:

@@ -154,6 +154,65 @@ combine_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict_
   }
 }
 
+// K <= KMAX: the K rows of a column chunk are loaded before any arithmetic, so
+// a warp keeps K*U 16-byte loads in flight.
+template <int U, int KMAX>
+__global__ void __launch_bounds__(kThreads)
+combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ y,
+                     const float *__restrict__ gates, uint4 *__restrict__ out, int64_t T, int K,
+                     int64_t nvec, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    int rows[KMAX];
+    float ws[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; k++) {
+      rows[k] = __shfl_sync(0xffffffffu, my_slot, k);
+      ws[k] = __shfl_sync(0xffffffffu, my_w, k);
+    }
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      uint4 q[KMAX][U];
+#pragma unroll
+      for (int k = 0; k < KMAX; k++)
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          q[k][u] = (rows[k] >= 0 && v < nvec) ? __ldcs(y + (int64_t)rows[k] * nvec + v)
+                                               : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < KMAX; k++) {
+          if (rows[k] < 0) continue;  // k >= K, or a pair without a slot
+          const uint32_t wd[4] = {q[k][u].x, q[k][u].y, q[k][u].z, q[k][u].w};
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            acc[2 * i] = __fmaf_rn(ws[k], bf16_lo(wd[i]), acc[2 * i]);
+            acc[2 * i + 1] = __fmaf_rn(ws[k], bf16_hi(wd[i]), acc[2 * i + 1]);
+          }
+        }
+        if (v < nvec) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[0], acc[1]);
+          o.y = pack_bf16x2(acc[2], acc[3]);
+          o.z = pack_bf16x2(acc[4], acc[5]);
+          o.w = pack_bf16x2(acc[6], acc[7]);
+          out[t * nvec + v] = o;
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads)
 combine_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ y,
                       const float *__restrict__ gates, uint16_t *__restrict__ out, int64_t T, int K,
@@ -234,6 +293,79 @@ combine_bwd_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restr
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
       if (lane == k) my_dg = part;
+    }
+    if (lane < K) dgates[t * K + lane] = my_dg;
+  }
+}
+
+// K <= KMAX: each dout row is read once.  For a column chunk the dout vectors
+// and the K expert-output vectors are loaded together; per-k dot partials stay
+// in registers until a warp tree reduces them at the end of the row.
+template <int U, int KMAX>
+__global__ void __launch_bounds__(kThreads)
+combine_bwd_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ dout,
+                         const uint4 *__restrict__ y, const float *__restrict__ gates,
+                         uint4 *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
+                         int64_t nvec, int64_t nrows, int32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t t = warp_g; t < T; t += nwarps) {
+    const int my_slot = load_slot(slot_of, t, K, nrows, status);
+    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    int rows[KMAX];
+    float ws[KMAX], part[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; k++) {
+      rows[k] = __shfl_sync(0xffffffffu, my_slot, k);
+      ws[k] = __shfl_sync(0xffffffffu, my_w, k);
+      part[k] = 0.f;
+    }
+    const uint4 *g = dout + t * nvec;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+      uint4 gq[U], yq[KMAX][U];
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        gq[u] = v < nvec ? __ldcs(g + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < KMAX; k++)
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          yq[k][u] = (rows[k] >= 0 && v < nvec) ? __ldcs(y + (int64_t)rows[k] * nvec + v)
+                                                : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int k = 0; k < KMAX; k++) {
+        if (rows[k] < 0) continue;
+        uint4 *dr = dy + (int64_t)rows[k] * nvec;
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          if (v >= nvec) continue;
+          const uint32_t gw[4] = {gq[u].x, gq[u].y, gq[u].z, gq[u].w};
+          const uint32_t yw[4] = {yq[k][u].x, yq[k][u].y, yq[k][u].z, yq[k][u].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+            part[k] = __fmaf_rn(g0, bf16_lo(yw[i]), part[k]);
+            part[k] = __fmaf_rn(g1, bf16_hi(yw[i]), part[k]);
+            o[i] = pack_bf16x2(__fmul_rn(ws[k], g0), __fmul_rn(ws[k], g1));
+          }
+          dr[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+    float my_dg = 0.f;
+#pragma unroll
+    for (int k = 0; k < KMAX; k++) {
+      float p = part[k];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+      if (lane == k) my_dg = p;
     }
     if (lane < K) dgates[t * K + lane] = my_dg;
   }
@@ -445,7 +577,11 @@ extern "C" moonep_status_t moonep_combine(const moonep_config_t *cfg, const void
   PlanPtrs P = plan_ptrs(d, plan_arena);
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS;
-  if (d.H % 8 == 0 && aligned16(y) && aligned16(out)) {
+  if (d.H % 8 == 0 && aligned16(y) && aligned16(out) && d.K <= 8) {
+    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
+        T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else if (d.H % 8 == 0 && aligned16(y) && aligned16(out)) {
     combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
         T, (int)d.K, d.H / 8, nrows, dev_status);
@@ -470,7 +606,12 @@ extern "C" moonep_status_t moonep_combine_backward(const moonep_config_t *cfg,
   PlanPtrs P = plan_ptrs(d, plan_arena);
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS;
-  if (d.H % 8 == 0 && aligned16(dout) && aligned16(y) && aligned16(dy)) {
+  const bool vec = d.H % 8 == 0 && aligned16(dout) && aligned16(y) && aligned16(dy);
+  if (vec && d.K <= 8) {
+    combine_bwd_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(dout), reinterpret_cast<const uint4 *>(y),
+        gates, reinterpret_cast<uint4 *>(dy), dgates, T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else if (vec) {
     combine_bwd_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(dout), reinterpret_cast<const uint4 *>(y),
         gates, reinterpret_cast<uint4 *>(dy), dgates, T, (int)d.K, d.H / 8, nrows, dev_status);

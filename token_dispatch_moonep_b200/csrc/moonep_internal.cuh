@@ -5,22 +5,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "moonep.h"
 
 namespace moonep {
 
-constexpr int kPlanThreads = 512;         // threads of the histogram / solve kernel
+constexpr int kPlanThreads = 512;   // threads per CTA of the plan kernel
 constexpr int kPlanWarps = kPlanThreads / 32;
-constexpr int kPairsPerThread = 16;        // pairs per thread in the histogram pass
-constexpr int kChunk = kPlanThreads * kPairsPerThread;  // pairs per histogram chunk (8192)
-constexpr int kPlaceThreads = 256;
-constexpr int kPlacePairsPerThread = 4;
-constexpr int kPlacePairsPerBlock = kPlaceThreads * kPlacePairsPerThread;
+constexpr int kPairsPerThread = 16;  // most pairs per thread in one plan chunk
 constexpr size_t kAlignBytes = 256;
 
 // ----------------------------------------------------------------- config ---
 struct Dims {
-  int64_t R, E, K, S, H, B, A, L, SK, N, NvS, NC, PMAX;
+  int64_t R, E, K, S, H, B, A, L, SK, N, NvS, NCMAX, PMAX;  // NCMAX: most plan chunks (512 pairs each)
   int mode;
 };
 
@@ -45,7 +43,7 @@ inline bool make_dims(const moonep_config_t *c, Dims *d) {
   d->N = d->R * d->SK;
   d->NvS = nvs_of(d->S, d->K, d->E, d->A);
   if (d->N >= (int64_t(1) << 31) || d->R * d->NvS >= (int64_t(1) << 31)) return false;
-  d->NC = d->N > 0 ? (d->N + kChunk - 1) / kChunk : 1;
+  d->NCMAX = d->N > 0 ? (d->N + kPlanThreads - 1) / kPlanThreads : 1;
   d->PMAX = d->E + d->R;
   return true;
 }
@@ -95,15 +93,26 @@ inline PlanPtrs plan_ptrs(const Dims &d, const void *arena) {
 }
 
 // -------------------------------------------------------------- workspace ---
-enum WsField { W_COUNTER, W_HIST, W_RANK, W_EXP_KEPT, W_EXP_ROW0, W_EXP_OSTART, W_PIECE_GROW, W_COUNT };
+// Plan scratch: sync words (generation, done, state, tables-done), per-chunk
+// arrival epochs (plus slots for diagnostic phantom arrivals), per-chunk
+// bad-id marks, per-chunk histograms, stable ranks, placement constants.
+constexpr int kSyncWords = 16;
+constexpr int kSyncMaxPhantom = 32;
+
+enum WsField {
+  W_SYNC, W_ARRIVE, W_BADMARK, W_HIST, W_RANK, W_EXP_KEPT, W_EXP_ROW0, W_EXP_OSTART, W_PIECE_GROW,
+  W_COUNT
+};
 
 struct WsLayout {
   size_t off[W_COUNT];
   size_t total;
   explicit WsLayout(const Dims &d) {
     const size_t n[W_COUNT] = {
-        8 * sizeof(int32_t),
-        size_t(d.E * d.NC) * sizeof(int32_t),
+        size_t(kSyncWords) * sizeof(int32_t),
+        size_t(d.NCMAX + kSyncMaxPhantom) * sizeof(int32_t),
+        size_t(d.NCMAX) * sizeof(int32_t),
+        size_t(d.E * d.NCMAX) * sizeof(int32_t),
         size_t(d.N > 0 ? d.N : 1) * sizeof(uint16_t),
         size_t(d.E) * sizeof(int32_t), size_t(d.E) * sizeof(int32_t), size_t(d.E) * sizeof(int32_t),
         size_t(d.PMAX) * sizeof(int32_t)};

@@ -3,18 +3,26 @@
 // duplicated onto underloaded ranks within a replica-slot budget;
 // "MoonshotAI/MoonEP 딥다이브" §4 pattern 1: planned once per layer, reused).
 //
-// Two kernels:
-//   plan_hist_solve  one CTA per chunk of 8192 (rank, token, k) pairs.  Each CTA
-//                    builds its chunk's per-expert histogram and the stable rank
-//                    of every pair among the chunk's pairs of the same expert
-//                    (warp-private counters + __match_any_sync, so a hot expert
-//                    never serialises on an atomic).  The last CTA to finish
-//                    (arrival counter; no CTA ever waits for another) scans the
-//                    histograms per expert into per-chunk bases and solves the
-//                    O(E + R) balance problem in shared memory.
-//   plan_place       every pair's final row: position inside its expert's list
-//                    = chunk base + stable rank; the first kept_e positions stay
-//                    in the home segment, the rest map through the piece table.
+// One cooperative kernel: CTA 0 solves, CTAs 1..W are workers.
+//   workers  take chunks of 512*ppt (rank, token, k) pairs (ppt <= 16, sized so
+//            that all SMs share the work).  Warp-private per-expert counters in
+//            shared memory give every pair its stable rank among the chunk's
+//            pairs of the same expert (lanes with equal ids are found with a
+//            shuffle-built peer mask: a hot expert costs one counter update per
+//            warp step, no atomics); the chunk histogram is published with an
+//            arrival flag.  While CTA 0 solves, each worker sums the histograms
+//            of the chunks before its own into its chunk's base offsets.
+//   CTA 0    waits for every arrival, sums the histograms into expert counts and
+//            solves the O(E + R) balance problem in shared memory.  It publishes
+//            the tables placement needs first (done flag), then writes the
+//            remaining plan tables while the workers place.
+//   workers  wait for the done flag and place their pairs: position in the
+//            expert's list = chunk base + stable rank; the first kept_e
+//            positions stay in the home segment, the rest map through the
+//            expert's pieces.
+// Flags carry a per-launch epoch derived from a generation word on the device,
+// so graph replays and reused workspaces need no memset; every wait is bounded
+// in time and reports MOONEP_DEV_TIMEOUT instead of hanging.
 #include <atomic>
 
 #include "moonep_internal.cuh"
@@ -23,40 +31,113 @@ namespace moonep {
 
 namespace {
 
+// process-wide diagnostics (moonep_debug_set_wait)
+std::atomic<long long> g_wait_limit_ns{200LL * 1000 * 1000};
+std::atomic<int> g_phantom_arrivals{0};
+
+constexpr int kStBad = 1, kStCapacity = 2, kStTimeout = 8;
+// Odd step between launch epochs: values left in a reused workspace (previous
+// epochs, constant fills, zeros) never equal the next epoch by accident.
+constexpr unsigned kEpochStep = 0x9E3779B1u;
+constexpr int kSyncGen = 0, kSyncDone = 1, kSyncState = 2, kSyncTables = 3;
+
+struct PlanArgs {
+  Dims d;
+  int ppt;        // pairs per thread of a chunk
+  int workers;    // CTAs 1..workers
+  int64_t ch;     // pairs per chunk (512 * ppt)
+  int64_t nc;     // chunks
+  const int32_t *idx;
+  PlanPtrs P;
+  int32_t *sync;     // generation, done, state, tables-done
+  int32_t *arrive;   // [nc + phantom] per-chunk arrival epochs
+  int32_t *badmark;  // [nc]
+  int32_t *hist;     // [nc][E] chunk histograms (rewritten as bases when chunks > workers)
+  uint16_t *rank;    // [N] stable ranks (only when a worker has several chunks)
+  int32_t *exp_kept, *exp_row0, *exp_ostart, *piece_grow;
+  int32_t *status;
+  long long wait_ns;
+  int phantom;
+};
+
 __device__ __forceinline__ int roundup_i(int v, int a) { return (v + a - 1) / a * a; }
 
-// Exclusive scan of s[0, n) in shared memory, in place; every thread of the block
-// calls it.  scratch: 33 ints of shared memory.  Returns the total.
-__device__ int block_excl_scan(int *s, int n, int *scratch) {
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int32_t *p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Warp-wide bounded wait until flags[0, n) all equal v.  False on timeout.
+__device__ bool warp_wait_all(const int32_t *flags, int64_t n, int v, long long limit_ns) {
+  const int lane = threadIdx.x & 31;
+  const unsigned long long t0 = now_ns();
+  int64_t from = 0;  // flags before `from` are known to have arrived
+  for (;;) {
+    bool mine = true;
+    for (int64_t c = from + lane; c < n && c < from + 1024; c += 32) mine &= ld_acquire(flags + c) == v;
+    if (__all_sync(0xffffffffu, mine)) {
+      from += 1024;
+      if (from >= n) return true;
+      continue;
+    }
+    if ((long long)(now_ns() - t0) > limit_ns) return false;
+    __nanosleep(64);
+  }
+}
+
+// Exclusive scans of NA arrays a[k][0, n) in shared memory, in place, one pass;
+// every thread of the block calls it.  scratch: 4*33 ints.  Totals in tot.
+template <int NA>
+__device__ void block_excl_scan(int *const (&a)[NA], int n, int *scratch, int (&tot)[NA]) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
   const int per = (n + nt - 1) / nt;
   const int b = tid * per < n ? tid * per : n;
   const int e = b + per < n ? b + per : n;
-  int sum = 0;
-  for (int i = b; i < e; i++) sum += s[i];
-  const int incl = warp_incl_scan(sum);
-  if (lane == 31) scratch[warp] = incl;
+  int sum[NA], incl[NA];
+#pragma unroll
+  for (int k = 0; k < NA; k++) {
+    sum[k] = 0;
+    for (int i = b; i < e; i++) sum[k] += a[k][i];
+    incl[k] = warp_incl_scan(sum[k]);
+    if (lane == 31) scratch[k * 33 + warp] = incl[k];
+  }
   __syncthreads();
   if (warp == 0) {
-    const int v = lane < nwarps ? scratch[lane] : 0;
-    const int wi = warp_incl_scan(v);
-    if (lane < nwarps) scratch[lane] = wi - v;
-    if (lane == 31) scratch[32] = wi;
+#pragma unroll
+    for (int k = 0; k < NA; k++) {
+      const int v = lane < nwarps ? scratch[k * 33 + lane] : 0;
+      const int wi = warp_incl_scan(v);
+      if (lane < nwarps) scratch[k * 33 + lane] = wi - v;
+      if (lane == 31) scratch[k * 33 + 32] = wi;
+    }
   }
   __syncthreads();
-  int run = scratch[warp] + incl - sum;
-  for (int i = b; i < e; i++) {
-    const int v = s[i];
-    s[i] = run;
-    run += v;
+#pragma unroll
+  for (int k = 0; k < NA; k++) {
+    int run = scratch[k * 33 + warp] + incl[k] - sum[k];
+    for (int i = b; i < e; i++) {
+      const int v = a[k][i];
+      a[k][i] = run;
+      run += v;
+    }
+    tot[k] = scratch[k * 33 + 32];
   }
-  const int total = scratch[32];
   __syncthreads();
-  return total;
 }
 
-// first index i in [0, n) with a[i] > v (n if none); a non-decreasing
+// first i in [0, n) with a[i] > v (n if none); a non-decreasing
 __device__ __forceinline__ int upper_bound_i(const int *a, int n, int v) {
   int lo = 0, hi = n;
   while (lo < hi) {
@@ -66,349 +147,64 @@ __device__ __forceinline__ int upper_bound_i(const int *a, int n, int v) {
   return lo;
 }
 
-// first index i in [0, n) with a[i] >= v
-__device__ __forceinline__ int lower_bound_i(const int *a, int n, int v) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (a[mid] >= v) hi = mid; else lo = mid + 1;
-  }
-  return lo;
-}
-
-// --------------------------------------------------------------- the solve --
-// Runs in the last CTA of plan_hist_solve.  hist[c*E + e] holds chunk c's
-// count of expert e on entry and the exclusive per-expert prefix on exit.
-__device__ void solve(const Dims &d, int *smem, PlanPtrs P, int32_t *wsflags, int32_t *hist,
-                      int32_t *exp_kept, int32_t *exp_row0, int32_t *exp_ostart,
-                      int32_t *piece_grow, int32_t *status) {
+// out[e] = sum of hist rows [0, nrows) at column e (E columns).  Rows are read
+// as 16-byte vectors when E % 4 == 0, many rows in flight per thread.
+// red: 4*blockDim.x ints of shared scratch.  Ends with __syncthreads().
+__device__ void column_sums(const int32_t *hist, int E, int64_t nrows, int *out, int *red) {
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, A = (int)d.A, B = (int)d.B;
-  const int SK = (int)d.SK, NvS = (int)d.NvS;
-  const int64_t NC = d.NC;
-  const int PMAX = (int)d.PMAX;
-
-  int *s = smem;
-  int *s_cnt = s; s += E;
-  int *s_cst = s; s += E;   // offset of the expert's list inside its home stream
-  int *s_kept = s; s += E;
-  int *s_ost = s; s += E;   // offset of the expert's first leaving entry in the overflow stream
-  int *s_npc = s; s += E;   // pieces of the expert
-  int *s_pbeg = s; s += E;  // first piece id of the expert
-  int *s_nst = s; s += E;   // start row of the expert's native segment within its rank
-  int *s_i0 = s; s += E;    // first receiver index of the expert's pieces
-  int *s_flag = s; s += E;  // expert has a local replica piece
-  int *s_load = s; s += R;
-  int *s_hbase = s; s += R;
-  int *s_over = s; s += R;
-  int *s_def = s; s += R;
-  int *s_obase = s; s += R;
-  int *s_dbase = s; s += R;
-  int *s_ridx = s; s += R;  // receiver index of a rank, -1 if it receives nothing
-  int *s_nbase = s; s += R;
-  int *s_ntot = s; s += R;  // rows used by the rank's native segments
-  int *s_rrank = s; s += R; // per receiver index i (< n_recv)
-  int *s_rbase = s; s += R;
-  int *s_rend = s; s += R;
-  int *s_rfirst = s; s += R;
-  int *s_rcount = s; s += R;
-  int *s_rpbase = s; s += R;
-  int *s_pexp = s; s += PMAX;
-  int *s_precv = s; s += PMAX;
-  int *s_post = s; s += PMAX;
-  int *s_plen = s; s += PMAX;
-  int *s_pj = s; s += PMAX;
-  int *s_pst = s; s += PMAX;
-  int *scratch = s; s += 40;  // [0..32] scan scratch, [33..39] block-wide values
-
-  const bool bad_ids = __ldcg(wsflags + 1) != 0;
-
-  // S1: per-expert exclusive scan over chunks; G lanes share one expert column.
-  {
-    int G = 1;
-    while (G < 32 && 2 * G * E <= nt) G *= 2;
-    const int grp = tid / G, sub = tid % G, ngrp = nt / G;
-    const int per = (int)((NC + G - 1) / G);
-    for (int e0 = 0; e0 < E; e0 += ngrp) {
-      const int e = e0 + grp;
-      const bool act = e < E;
-      const int c0 = sub * per;
-      const int c1 = (int)(c0 + per < NC ? c0 + per : NC);
-      int sum = 0;
-      if (act) {
-        int c = c0;
-        for (; c + 16 <= c1; c += 16) {
-          int v[16];
+  if ((E & 3) == 0 && E / 4 <= nt) {
+    const int E4 = E / 4, groups = nt / E4;
+    const int g = tid / E4, col = tid % E4;
+    int4 acc = make_int4(0, 0, 0, 0);
+    if (g < groups) {
+      const int4 *h4 = reinterpret_cast<const int4 *>(hist);
+      for (int64_t r0 = g; r0 < nrows; r0 += (int64_t)groups * 8) {
+        int4 v[8];
 #pragma unroll
-          for (int u = 0; u < 16; u++) v[u] = __ldcg(hist + (int64_t)(c + u) * E + e);
-#pragma unroll
-          for (int u = 0; u < 16; u++) sum += v[u];
+        for (int u = 0; u < 8; u++) {
+          const int64_t r = r0 + (int64_t)u * groups;
+          v[u] = r < nrows ? __ldcg(h4 + r * E4 + col) : make_int4(0, 0, 0, 0);
         }
-        for (; c < c1; c++) sum += __ldcg(hist + (int64_t)c * E + e);
-      }
-      // exclusive scan of the G partial sums inside the group
-      int incl = sum;
-      for (int o = 1; o < G; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o, G);
-        if (sub >= o) incl += n;
-      }
-      int run = incl - sum;
-      const int total = __shfl_sync(0xffffffffu, incl, G - 1, G);
-      if (act) {
-        int c = c0;
-        for (; c + 16 <= c1; c += 16) {
-          int v[16];
 #pragma unroll
-          for (int u = 0; u < 16; u++) v[u] = __ldcg(hist + (int64_t)(c + u) * E + e);
-#pragma unroll
-          for (int u = 0; u < 16; u++) {
-            hist[(int64_t)(c + u) * E + e] = run;
-            run += v[u];
-          }
+        for (int u = 0; u < 8; u++) {
+          acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
         }
-        for (; c < c1; c++) {
-          const int v = __ldcg(hist + (int64_t)c * E + e);
-          hist[(int64_t)c * E + e] = run;
-          run += v;
-        }
-        if (sub == 0) s_cnt[e] = total;
       }
+      reinterpret_cast<int4 *>(red)[g * E4 + col] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += nt) {
+      int s = 0;
+      for (int q = 0; q < groups; q++) s += red[q * E + e];
+      out[e] = s;
+    }
+  } else {
+    for (int e = tid; e < E; e += nt) {
+      int s = 0;
+      for (int64_t r = 0; r < nrows; r++) s += __ldcg(hist + r * E + e);
+      out[e] = s;
     }
   }
   __syncthreads();
-
-  // S2: rank loads and each expert's offset inside its home stream
-  for (int e = tid; e < E; e += nt) s_cst[e] = s_cnt[e];
-  __syncthreads();
-  const int total_pairs = block_excl_scan(s_cst, E, scratch);
-  for (int h = tid; h < R; h += nt) {
-    const int lo = s_cst[h * L];
-    const int hi = (h + 1) * L < E ? s_cst[(h + 1) * L] : total_pairs;
-    s_hbase[h] = lo;
-    s_load[h] = hi - lo;
-    s_over[h] = hi - lo > SK ? hi - lo - SK : 0;
-    s_def[h] = hi - lo < SK ? SK - (hi - lo) : 0;
-    s_obase[h] = s_over[h];
-    s_dbase[h] = s_def[h];
-    s_ridx[h] = s_def[h] > 0 ? 1 : 0;
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += nt) s_cst[e] -= s_hbase[e / L];
-  block_excl_scan(s_obase, R, scratch);
-  block_excl_scan(s_dbase, R, scratch);
-  const int n_recv = block_excl_scan(s_ridx, R, scratch);
-  for (int h = tid; h < R; h += nt) {
-    if (s_def[h] > 0) {
-      const int i = s_ridx[h];
-      s_rrank[i] = h;
-      s_rbase[i] = s_dbase[h];
-      s_rend[i] = s_dbase[h] + s_def[h];
-      s_rfirst[i] = 0;
-      s_rcount[i] = 0;
-    } else {
-      s_ridx[h] = -1;
-    }
-  }
-  __syncthreads();
-
-  // S3: kept rows, overflow position and piece count of every expert
-  for (int e = tid; e < E; e += nt) {
-    const int cnt = s_cnt[e], cst = s_cst[e], h = e / L;
-    int kept = SK - cst;
-    kept = kept < 0 ? 0 : (kept > cnt ? cnt : kept);
-    const int ovf = cnt - kept;
-    const int ost = s_obase[h] + (cst > SK ? cst - SK : 0);
-    s_kept[e] = kept;
-    s_ost[e] = ost;
-    int npc = 0, i0 = 0;
-    if (ovf > 0 && !bad_ids && n_recv > 0) {
-      i0 = upper_bound_i(s_rend, n_recv, ost);
-      int i1 = lower_bound_i(s_rend, n_recv, ost + ovf);
-      if (i1 >= n_recv) i1 = n_recv - 1;
-      if (i0 < n_recv) npc = i1 - i0 + 1;
-    }
-    s_npc[e] = npc;
-    s_pbeg[e] = npc;
-    s_i0[e] = i0;
-    s_nst[e] = roundup_i(kept, A);
-  }
-  __syncthreads();
-  int n_piece = block_excl_scan(s_pbeg, E, scratch);
-  if (n_piece > PMAX) n_piece = PMAX;  // cannot happen: pieces <= experts + receivers - 1
-  const int native_rows = block_excl_scan(s_nst, E, scratch);
-  for (int h = tid; h < R; h += nt) {
-    const int lo = s_nst[h * L];
-    const int hi = (h + 1) * L < E ? s_nst[(h + 1) * L] : native_rows;
-    s_nbase[h] = lo;
-    s_ntot[h] = hi - lo;
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += nt) s_nst[e] -= s_nbase[e / L];
-
-  // S4: pieces = intersections of expert overflow ranges with receiver ranges
-  for (int e = tid; e < E; e += nt) {
-    const int npc = s_npc[e];
-    if (npc == 0) continue;
-    const int ost = s_ost[e], oend = ost + (s_cnt[e] - s_kept[e]);
-    for (int q = 0; q < npc; q++) {
-      const int i = s_i0[e] + q, pid = s_pbeg[e] + q;
-      if (pid >= PMAX) break;
-      const int os = ost > s_rbase[i] ? ost : s_rbase[i];
-      const int oe = oend < s_rend[i] ? oend : s_rend[i];
-      s_pexp[pid] = e;
-      s_precv[pid] = i;
-      s_post[pid] = os;
-      s_plen[pid] = oe - os;
-      if (os == s_rbase[i]) s_rfirst[i] = pid;
-    }
-  }
-  __syncthreads();
-  for (int pid = tid; pid < n_piece; pid += nt) {
-    const int i = s_precv[pid];
-    const int j = pid - s_rfirst[i];
-    s_pj[pid] = j;
-    if (s_post[pid] + s_plen[pid] == s_rend[i]) s_rcount[i] = j + 1;
-    s_pst[pid] = roundup_i(s_plen[pid], A);
-  }
-  __syncthreads();
-  block_excl_scan(s_pst, n_piece, scratch);
-  for (int i = tid; i < n_recv; i += nt) s_rpbase[i] = s_pst[s_rfirst[i]];
-  if (tid == 0) { scratch[33] = 0; scratch[34] = 0; scratch[35] = 0; scratch[36] = 0; }
-  __syncthreads();
-  for (int pid = tid; pid < n_piece; pid += nt) {
-    const int i = s_precv[pid];
-    s_pst[pid] = s_ntot[s_rrank[i]] + s_pst[pid] - s_rpbase[i];
-  }
-  __syncthreads();
-
-  // capacity: every rank's rows must end inside NvS (true by construction)
-  for (int h = tid; h < R; h += nt) {
-    int used = s_ntot[h];
-    const int i = s_ridx[h];
-    if (i >= 0 && s_rcount[i] > 0) {
-      const int last = s_rfirst[i] + s_rcount[i] - 1;
-      used = s_pst[last] + s_plen[last];
-    }
-    if (used > NvS) atomicOr(&scratch[33], 1);
-  }
-  // remote pieces and experts with a local replica
-  for (int e = tid; e < E; e += nt) s_flag[e] = 0;
-  __syncthreads();
-  for (int pid = tid; pid < n_piece; pid += nt) {
-    if (s_pj[pid] >= B) atomicAdd(&scratch[34], 1);
-    else s_flag[s_pexp[pid]] = 1;
-  }
-  __syncthreads();
-  const bool capacity_bad = scratch[33] != 0;
-  const int n_remote = scratch[34];
-  // compact list of experts with a local replica (ascending)
-  for (int e = tid; e < E; e += nt) s_i0[e] = s_flag[e];
-  __syncthreads();
-  const int n_replicated = block_excl_scan(s_i0, E, scratch);
-
-  // S5: outputs
-  int32_t *o_count = P.f[F_EXPERT_COUNT];
-  for (int e = tid; e < E; e += nt) {
-    const int h = e / L;
-    o_count[e] = s_cnt[e];
-    P.f[F_EXP_PIECE_BEGIN][e] = s_pbeg[e];
-    P.f[F_EXP_PIECE_END][e] = s_pbeg[e] + s_npc[e];
-    exp_kept[e] = s_kept[e];
-    exp_row0[e] = h * NvS + s_nst[e];
-    exp_ostart[e] = s_ost[e];
-    const int si = h * E + (e - h * L);
-    P.f[F_SEG_EXPERT][si] = e;
-    P.f[F_SEG_START][si] = s_nst[e];
-    P.f[F_SEG_LEN][si] = s_kept[e];
-    P.f[F_SEG_KIND][si] = MOONEP_SEG_NATIVE;
-    P.f[F_SEG_WSLOT][si] = -1;
-    if (s_flag[e]) P.f[F_REPLICATED][s_i0[e]] = e;
-  }
-  for (int h = tid; h < R; h += nt) {
-    P.f[F_RANK_LOAD][h] = s_load[h];
-    P.f[F_OVERFLOW][h] = s_over[h];
-    P.f[F_DEFICIT][h] = s_def[h];
-    const int i = s_ridx[h];
-    P.f[F_N_SEG][h] = L + (i >= 0 ? s_rcount[i] : 0);
-  }
-  for (int pid = tid; pid < n_piece; pid += nt) {
-    const int i = s_precv[pid], dr = s_rrank[i], j = s_pj[pid];
-    const int e = s_pexp[pid];
-    const int ws = j < B ? j : -1;
-    P.f[F_PIECE_EXPERT][pid] = e;
-    P.f[F_PIECE_RANK][pid] = dr;
-    P.f[F_PIECE_START][pid] = s_pst[pid];
-    P.f[F_PIECE_LEN][pid] = s_plen[pid];
-    P.f[F_PIECE_WSLOT][pid] = ws;
-    P.f[F_PIECE_OSTART][pid] = s_post[pid];
-    piece_grow[pid] = dr * NvS + s_pst[pid];
-    if (L + j < E) {
-      const int si = dr * E + L + j;
-      P.f[F_SEG_EXPERT][si] = e;
-      P.f[F_SEG_START][si] = s_pst[pid];
-      P.f[F_SEG_LEN][si] = s_plen[pid];
-      P.f[F_SEG_KIND][si] = ws >= 0 ? MOONEP_SEG_REPLICA : MOONEP_SEG_REMOTE;
-      P.f[F_SEG_WSLOT][si] = ws;
-    }
-  }
-  for (int64_t q = tid; q < d.R * d.E; q += nt) {
-    const int h = (int)(q / E), i = (int)(q % E);
-    const int ri = s_ridx[h];
-    const int nseg = L + (ri >= 0 ? s_rcount[ri] : 0);
-    if (i >= nseg) {
-      P.f[F_SEG_EXPERT][q] = -1;
-      P.f[F_SEG_START][q] = 0;
-      P.f[F_SEG_LEN][q] = 0;
-      P.f[F_SEG_KIND][q] = -1;
-      P.f[F_SEG_WSLOT][q] = -1;
-    }
-  }
-  for (int64_t q = tid; q < d.R * d.B; q += nt) {
-    const int h = (int)(q / B), j = (int)(q % B);
-    const int ri = s_ridx[h];
-    P.f[F_REP_EXPERT][q] = (ri >= 0 && j < s_rcount[ri]) ? s_pexp[s_rfirst[ri] + j] : -1;
-  }
-  if (tid == 0) {
-    int32_t *sc = P.f[F_SCALARS];
-    sc[S_N_PIECE] = n_piece;
-    sc[S_N_REMOTE] = n_remote;
-    sc[S_N_LOCAL] = n_piece - n_remote;
-    sc[S_N_REPLICATED] = n_replicated;
-    sc[S_BAD] = (bad_ids ? 1 : 0) | (capacity_bad ? 2 : 0);
-    sc[5] = sc[6] = sc[7] = 0;
-    if (capacity_bad) {
-      wsflags[2] = 1;
-      set_status(status, MOONEP_DEV_CAPACITY);
-    }
-    if (d.mode == MOONEP_MODE_TRAIN && n_remote > 0) set_status(status, MOONEP_DEV_BUDGET);
-  }
 }
 
-// ----------------------------------------------------- histogram + solve ---
-__global__ void __launch_bounds__(kPlanThreads)
-plan_hist_solve_kernel(Dims d, const int32_t *__restrict__ idx, PlanPtrs P, int32_t *wsflags,
-                       int32_t *hist, uint16_t *rank_out, int32_t *exp_kept, int32_t *exp_row0,
-                       int32_t *exp_ostart, int32_t *piece_grow, int32_t *status) {
-  extern __shared__ int smem[];
-  __shared__ int s_last;
+// ------------------------------------------------------- worker counting ---
+// Histogram of chunk k and the stable rank of each of its pairs among the
+// chunk's pairs of the same expert.  Pair of (warp w, step j, lane l) is
+// k*ch + w*32*ppt + j*32 + l.  ev[j]: expert id, -1 bad id, -2 past the end.
+__device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *wh,
+                                            int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int E = (int)d.E;
-  const int64_t c = blockIdx.x;
-
-  int *wh = smem;  // [kPlanWarps][E] warp-private running counts
+  const int E = (int)a.d.E, ppt = a.ppt;
   for (int i = tid; i < kPlanWarps * E; i += kPlanThreads) wh[i] = 0;
-  __syncthreads();
-
-  const int64_t base = c * kChunk + (int64_t)warp * (32 * kPairsPerThread);
-  int ev[kPairsPerThread];
-  int rk[kPairsPerThread];
+  const int64_t base = k * a.ch + (int64_t)warp * 32 * ppt;
   bool bad = false;
 #pragma unroll
   for (int j = 0; j < kPairsPerThread; j++) {
     const int64_t p = base + j * 32 + lane;
-    int e = -2;  // past the end
-    if (p < d.N) {
-      e = __ldcs(idx + p);
+    int e = -2;
+    if (j < ppt && p < a.d.N) {
+      e = __ldcs(a.idx + p);
       if (e < 0 || e >= E) {
         bad = true;
         e = -1;
@@ -416,123 +212,567 @@ plan_hist_solve_kernel(Dims d, const int32_t *__restrict__ idx, PlanPtrs P, int3
     }
     ev[j] = e;
   }
+  __syncthreads();
   int *myh = wh + warp * E;
+  const uint32_t lt = lanemask_lt();
 #pragma unroll
   for (int j = 0; j < kPairsPerThread; j++) {
+    if (j >= ppt) break;  // uniform across the block
     const int e = ev[j];
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    uint32_t peers = 0;
+#pragma unroll
+    for (int l = 0; l < 32; l++) peers |= (uint32_t)(__shfl_sync(0xffffffffu, e, l) == e) << l;
     const int prev = e >= 0 ? myh[e] : 0;
-    const int r = __popc(peers & lanemask_lt());
+    const int r = __popc(peers & lt);
     rk[j] = prev + r;
     __syncwarp();
     if (e >= 0 && r == 0) myh[e] = prev + __popc(peers);
     __syncwarp();
   }
-  if (bad) {
-    set_status(status, MOONEP_DEV_BAD_EXPERT_ID);
-    atomicOr(wsflags + 1, 1);
-  }
   __syncthreads();
-  // per expert: exclusive prefix over warps, chunk total
   for (int e = tid; e < E; e += kPlanThreads) {
     int acc = 0;
+#pragma unroll
     for (int w = 0; w < kPlanWarps; w++) {
       const int v = wh[w * E + e];
       wh[w * E + e] = acc;
       acc += v;
     }
-    hist[c * E + e] = acc;
+    a.hist[k * E + e] = acc;
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < kPairsPerThread; j++) {
-    const int64_t p = base + j * 32 + lane;
-    if (ev[j] >= 0) rank_out[p] = (uint16_t)(myh[ev[j]] + rk[j]);
-  }
-
-  // arrival: the last CTA solves (nobody waits)
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(wsflags, 1) == (int)gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  solve(d, smem, P, wsflags, hist, exp_kept, exp_row0, exp_ostart, piece_grow, status);
+  for (int j = 0; j < kPairsPerThread; j++)
+    if (ev[j] >= 0) rk[j] += myh[ev[j]];
+  __syncthreads();  // wh is reused by the caller
+  return bad;
 }
 
-// ---------------------------------------------------------------- placing ---
-__global__ void __launch_bounds__(kPlaceThreads)
-plan_place_kernel(Dims d, const int32_t *__restrict__ idx, PlanPtrs P, const int32_t *wsflags,
-                  const int32_t *__restrict__ hist, const uint16_t *__restrict__ rank_in,
-                  const int32_t *__restrict__ exp_kept, const int32_t *__restrict__ exp_row0,
-                  const int32_t *__restrict__ exp_ostart, const int32_t *__restrict__ piece_grow) {
-  const bool invalid = (wsflags[1] | wsflags[2]) != 0;
-  const int E = (int)d.E;
-  int32_t *slot_of = P.f[F_SLOT_OF];
-  int32_t *slot_src = P.f[F_SLOT_SRC];
-  const int32_t *pbeg = P.f[F_EXP_PIECE_BEGIN];
-  const int32_t *pend = P.f[F_EXP_PIECE_END];
-  const int32_t *post = P.f[F_PIECE_OSTART];
-  const int64_t nrows = d.R * d.NvS;
-  const int64_t p0 = (int64_t)blockIdx.x * kPlacePairsPerBlock + threadIdx.x;
+// ------------------------------------------------------------ the solve ---
+struct SolveSmem {
+  int *cnt, *cst, *kept, *ovf, *oend, *npc, *nst, *i0, *flag, *npcn;  // [E]
+  int *load, *over, *def, *ridx, *ntot, *nseg, *rrank, *rbase, *rend, *rfirst, *tmp;  // [R]
+  int *pexp, *precv, *post, *plen, *pst;  // [PMAX]
+  int *scratch, *misc, *red;  // 4*33, 8, 4*kPlanThreads
+};
+
+__device__ __forceinline__ SolveSmem carve(const Dims &d, int *s) {
+  const int E = (int)d.E, R = (int)d.R, PM = (int)d.PMAX;
+  SolveSmem m;
+  int **ea[10] = {&m.cnt, &m.cst, &m.kept, &m.ovf, &m.oend, &m.npc, &m.nst, &m.i0, &m.flag, &m.npcn};
+  for (int i = 0; i < 10; i++) { *ea[i] = s; s += E; }
+  int **ra[11] = {&m.load, &m.over, &m.def, &m.ridx, &m.ntot, &m.nseg, &m.rrank, &m.rbase, &m.rend,
+                  &m.rfirst, &m.tmp};
+  for (int i = 0; i < 11; i++) { *ra[i] = s; s += R; }
+  int **pa[5] = {&m.pexp, &m.precv, &m.post, &m.plen, &m.pst};
+  for (int i = 0; i < 5; i++) { *pa[i] = s; s += PM; }
+  m.scratch = s; s += 4 * 33;
+  m.misc = s; s += 8;
+  s = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(s) + 15) & ~uintptr_t(15));
+  m.red = s;
+  return m;
+}
+
+__host__ __device__ inline size_t solve_smem_ints(const Dims &d) {
+  return 10 * d.E + 11 * d.R + 5 * d.PMAX + 4 * 33 + 8 + 4 + 4 * kPlanThreads;
+}
+
+// Per-expert exclusive scan of the histograms over chunks, in place (the
+// bases of chunks when workers hold several chunks); counts into cnt.
+__device__ void chunk_bases(const PlanArgs &a, int *cnt) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int E = (int)a.d.E;
+  const int64_t NC = a.nc;
+  for (int e = tid; e < E; e += nt) {
+    int run = 0;
+    for (int64_t c = 0; c < NC; c += 16) {
+      int v[16];
 #pragma unroll
-  for (int j = 0; j < kPlacePairsPerThread; j++) {
-    const int64_t p = p0 + j * kPlaceThreads;
-    if (p >= d.N) break;
-    if (invalid) {
-      slot_of[p] = -1;
-      continue;
+      for (int u = 0; u < 16; u++) v[u] = c + u < NC ? __ldcg(a.hist + (c + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 16; u++) {
+        if (c + u < NC) a.hist[(c + u) * E + e] = run;
+        run += v[u];
+      }
     }
-    const int e = __ldcs(idx + p);
-    const int pos = hist[(p / kChunk) * E + e] + rank_in[p];
-    const int kept = exp_kept[e];
+    cnt[e] = run;
+  }
+  __syncthreads();
+}
+
+// The part of the solve placement depends on.  Returns state bits (thread 0).
+__device__ int solve_core(const PlanArgs &a, const SolveSmem &m) {
+  const Dims &d = a.d;
+  const PlanPtrs &P = a.P;
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, A = (int)d.A;
+  const int SK = (int)d.SK, NvS = (int)d.NvS, PM = (int)d.PMAX;
+
+  // rank loads from the global prefix of counts
+  for (int e = tid; e < E; e += nt) m.cst[e] = m.cnt[e];
+  if (tid == 0) { m.misc[1] = 0; m.misc[2] = 0; }
+  {
+    int *arr[1] = {m.cst};
+    int tot[1];
+    __syncthreads();
+    block_excl_scan<1>(arr, E, m.scratch, tot);
+    for (int h = tid; h < R; h += nt) {
+      const int lo = m.cst[h * L];
+      m.load[h] = ((h + 1) * L < E ? m.cst[(h + 1) * L] : tot[0]) - lo;
+    }
+  }
+  __syncthreads();
+  // overflow / deficit bases, receiver compaction
+  if (R <= 32) {
+    if (warp == 0) {
+      const int ld = lane < R ? m.load[lane] : SK;
+      const int ov = ld > SK ? ld - SK : 0;
+      const int df = ld < SK ? SK - ld : 0;
+      const int rf = df > 0 ? 1 : 0;
+      const int iov = warp_incl_scan(ov), idf = warp_incl_scan(df), irf = warp_incl_scan(rf);
+      if (lane < R) {
+        m.over[lane] = iov - ov;
+        m.def[lane] = idf - df;
+        m.ridx[lane] = rf ? irf - 1 : -1;
+        if (rf) {
+          m.rrank[irf - 1] = lane;
+          m.rbase[irf - 1] = idf - df;
+          m.rend[irf - 1] = idf;
+        }
+      }
+      if (lane == 31) m.misc[0] = irf;
+    }
+  } else {
+    for (int h = tid; h < R; h += nt) {
+      const int ld = m.load[h];
+      m.over[h] = ld > SK ? ld - SK : 0;
+      m.def[h] = ld < SK ? SK - ld : 0;
+      m.tmp[h] = m.def[h];
+      m.ridx[h] = m.def[h] > 0 ? 1 : 0;
+    }
+    int *arr[3] = {m.over, m.def, m.ridx};
+    int tot[3];
+    __syncthreads();
+    block_excl_scan<3>(arr, R, m.scratch, tot);
+    for (int h = tid; h < R; h += nt) {
+      if (m.tmp[h] > 0) {
+        const int i = m.ridx[h];
+        m.rrank[i] = h;
+        m.rbase[i] = m.def[h];
+        m.rend[i] = m.def[h] + m.tmp[h];
+      } else {
+        m.ridx[h] = -1;
+      }
+    }
+    if (tid == 0) m.misc[0] = tot[2];
+  }
+  __syncthreads();
+  const int n_recv = m.misc[0];
+
+  // per expert: kept rows, overflow range, pieces
+  for (int e = tid; e < E; e += nt) {
+    const int h = e / L;
+    const int cnt = m.cnt[e];
+    const int cst = m.cst[e] - m.cst[h * L];
+    int kept = SK - cst;
+    kept = kept < 0 ? 0 : (kept > cnt ? cnt : kept);
+    const int ovf = cnt - kept;
+    const int ost = m.over[h] + (cst > SK ? cst - SK : 0);
+    m.kept[e] = kept;
+    m.ovf[e] = ovf;
+    m.oend[e] = ost + ovf;
+    int npc = 0, i0 = 0;
+    if (ovf > 0 && n_recv > 0) {
+      i0 = upper_bound_i(m.rend, n_recv, ost);
+      int i1 = upper_bound_i(m.rend, n_recv, ost + ovf - 1);
+      if (i1 >= n_recv) i1 = n_recv - 1;
+      if (i0 < n_recv) npc = i1 - i0 + 1;
+    }
+    m.npc[e] = npc;
+    m.npcn[e] = npc;
+    m.i0[e] = i0;
+    m.nst[e] = A > 1 ? roundup_i(kept, A) : (cst < SK ? cst : SK);  // A = 1: kept rows are a prefix
+  }
+  int n_piece;
+  __syncthreads();
+  if (A > 1) {
+    int *arr[2] = {m.npc, m.nst};
+    int tot[2];
+    block_excl_scan<2>(arr, E, m.scratch, tot);
+    n_piece = tot[0];
+    for (int h = tid; h < R; h += nt) {
+      const int lo = m.nst[h * L];
+      m.ntot[h] = ((h + 1) * L < E ? m.nst[(h + 1) * L] : tot[1]) - lo;
+      m.tmp[h] = lo;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += nt) m.nst[e] -= m.tmp[e / L];
+  } else {
+    int *arr[1] = {m.npc};
+    int tot[1];
+    block_excl_scan<1>(arr, E, m.scratch, tot);
+    n_piece = tot[0];
+    for (int h = tid; h < R; h += nt) m.ntot[h] = m.load[h] < SK ? m.load[h] : SK;
+  }
+  if (n_piece > PM) n_piece = PM;  // cannot happen: pieces <= experts + receivers - 1
+  if (tid == 0) m.misc[3] = n_piece;
+  __syncthreads();
+
+  // placement tables
+  for (int e = tid; e < E; e += nt) {
+    const int h = e / L;
+    const int pb = m.npc[e], npc = m.npcn[e];
+    const int ost = m.oend[e] - m.ovf[e];
+    a.exp_kept[e] = m.kept[e];
+    a.exp_row0[e] = h * NvS + m.nst[e];
+    a.exp_ostart[e] = ost;
+    P.f[F_EXP_PIECE_BEGIN][e] = pb;
+    P.f[F_EXP_PIECE_END][e] = pb + npc;
+    for (int q = 0; q < npc; q++) {
+      const int i = m.i0[e] + q, pid = pb + q;
+      if (pid >= PM || i >= n_recv) break;
+      const int os = ost > m.rbase[i] ? ost : m.rbase[i];
+      const int oe = m.oend[e] < m.rend[i] ? m.oend[e] : m.rend[i];
+      const int dr = m.rrank[i];
+      int start;
+      if (A == 1) {
+        start = m.ntot[dr] + (os - m.rbase[i]);
+      } else {  // earlier pieces of receiver i: from the expert holding rbase up to e-1
+        const int ef = upper_bound_i(m.oend, E, m.rbase[i]);
+        start = m.ntot[dr];
+        if (ef < e) {
+          start += roundup_i(m.oend[ef] - m.rbase[i], A);
+          for (int e2 = ef + 1; e2 < e; e2++) start += roundup_i(m.ovf[e2], A);
+        }
+      }
+      m.pexp[pid] = e;
+      m.precv[pid] = i;
+      m.post[pid] = os;
+      m.plen[pid] = oe - os;
+      m.pst[pid] = start;
+      P.f[F_PIECE_OSTART][pid] = os;
+      a.piece_grow[pid] = dr * NvS + start;
+      if (start + (oe - os) > NvS) m.misc[1] = 1;
+    }
+  }
+  for (int h = tid; h < R; h += nt)
+    if (m.ntot[h] > NvS) m.misc[1] = 1;
+  __syncthreads();
+  return m.misc[1] ? kStCapacity : 0;
+}
+
+// Every other plan table (after the done flag; placement does not read them).
+__device__ void solve_outputs(const PlanArgs &a, const SolveSmem &m) {
+  const Dims &d = a.d;
+  const PlanPtrs &P = a.P;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
+  const int n_recv = m.misc[0], n_piece = m.misc[3];
+
+  for (int i = tid; i < n_recv; i += nt) {  // first and last piece of each receiver
+    const int ef = upper_bound_i(m.oend, E, m.rbase[i]);
+    m.rfirst[i] = ef < E ? m.npc[ef] + (i - m.i0[ef]) : 0;
+    const int el = upper_bound_i(m.oend, E, m.rend[i] - 1);
+    const int last = el < E ? m.npc[el] + (i - m.i0[el]) : -1;
+    m.nseg[m.rrank[i]] = L + (last - m.rfirst[i] + 1);
+  }
+  for (int h = tid; h < R; h += nt)
+    if (m.ridx[h] < 0) m.nseg[h] = L;
+  for (int e = tid; e < E; e += nt) m.flag[e] = 0;
+  __syncthreads();
+  for (int pid = tid; pid < n_piece; pid += nt) {
+    const int i = m.precv[pid], e = m.pexp[pid];
+    const int dr = m.rrank[i], j = pid - m.rfirst[i];
+    const int ws = j < B ? j : -1;
+    P.f[F_PIECE_EXPERT][pid] = e;
+    P.f[F_PIECE_RANK][pid] = dr;
+    P.f[F_PIECE_START][pid] = m.pst[pid];
+    P.f[F_PIECE_LEN][pid] = m.plen[pid];
+    P.f[F_PIECE_WSLOT][pid] = ws;
+    if (j >= 0 && L + j < E) {
+      const int sj = dr * E + L + j;
+      P.f[F_SEG_EXPERT][sj] = e;
+      P.f[F_SEG_START][sj] = m.pst[pid];
+      P.f[F_SEG_LEN][sj] = m.plen[pid];
+      P.f[F_SEG_KIND][sj] = ws >= 0 ? MOONEP_SEG_REPLICA : MOONEP_SEG_REMOTE;
+      P.f[F_SEG_WSLOT][sj] = ws;
+    }
+    if (ws >= 0) {
+      P.f[F_REP_EXPERT][(int64_t)dr * B + j] = e;
+      m.flag[e] = 1;
+    } else {
+      atomicAdd(&m.misc[2], 1);
+    }
+  }
+  for (int e = tid; e < E; e += nt) {
+    const int h = e / L, si = h * E + (e - h * L);
+    P.f[F_EXPERT_COUNT][e] = m.cnt[e];
+    P.f[F_SEG_EXPERT][si] = e;
+    P.f[F_SEG_START][si] = m.nst[e];
+    P.f[F_SEG_LEN][si] = m.kept[e];
+    P.f[F_SEG_KIND][si] = MOONEP_SEG_NATIVE;
+    P.f[F_SEG_WSLOT][si] = -1;
+  }
+  for (int h = tid; h < R; h += nt) {
+    const int ld = m.load[h];
+    P.f[F_RANK_LOAD][h] = ld;
+    P.f[F_OVERFLOW][h] = ld > SK ? ld - SK : 0;
+    P.f[F_DEFICIT][h] = ld < SK ? SK - ld : 0;
+    P.f[F_N_SEG][h] = m.nseg[h];
+  }
+  for (int64_t q = tid; q < d.R * d.E; q += nt) {  // unused segment entries
+    const int h = (int)(q / E), i = (int)(q % E);
+    if (i >= m.nseg[h]) {
+      P.f[F_SEG_EXPERT][q] = -1;
+      P.f[F_SEG_START][q] = 0;
+      P.f[F_SEG_LEN][q] = 0;
+      P.f[F_SEG_KIND][q] = -1;
+      P.f[F_SEG_WSLOT][q] = -1;
+    }
+  }
+  for (int64_t q = tid; q < d.R * d.B; q += nt) {  // free replica slots
+    const int h = (int)(q / B), j = (int)(q % B);
+    if (j >= m.nseg[h] - L) P.f[F_REP_EXPERT][q] = -1;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += nt) m.i0[e] = m.flag[e];  // keep the flags across the scan
+  {
+    int *arr[1] = {m.flag};
+    int tot[1];
+    __syncthreads();
+    block_excl_scan<1>(arr, E, m.scratch, tot);
+    for (int e = tid; e < E; e += nt)
+      if (m.i0[e]) P.f[F_REPLICATED][m.flag[e]] = e;
+    if (tid == 0) m.misc[4] = tot[0];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const int n_remote = m.misc[2];
+    int32_t *sc = P.f[F_SCALARS];
+    sc[S_N_PIECE] = n_piece;
+    sc[S_N_REMOTE] = n_remote;
+    sc[S_N_LOCAL] = n_piece - n_remote;
+    sc[S_N_REPLICATED] = m.misc[4];
+    sc[S_BAD] = 0;
+    sc[5] = sc[6] = sc[7] = 0;
+    if (d.mode == MOONEP_MODE_TRAIN && n_remote > 0) set_status(a.status, MOONEP_DEV_BUDGET);
+  }
+}
+
+// -------------------------------------------------------------- placing ---
+// tables: base[E] kept[E] row0[E] ostart[E] piece_begin[E] piece_end[E]
+//         piece_ostart[PMAX] piece_row[PMAX]
+__device__ __forceinline__ void place_chunk(const PlanArgs &a, int64_t k, const int *t, bool from_regs,
+                                            const int (&ev)[kPairsPerThread],
+                                            const int (&rk)[kPairsPerThread]) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Dims &d = a.d;
+  const int E = (int)d.E, PM = (int)d.PMAX, ppt = a.ppt;
+  const int *t_base = t, *t_kept = t + E, *t_row0 = t + 2 * E, *t_ost = t + 3 * E;
+  const int *t_pb = t + 4 * E, *t_pe = t + 5 * E, *t_post = t + 6 * E, *t_prow = t + 6 * E + PM;
+  int32_t *slot_of = a.P.f[F_SLOT_OF];
+  int32_t *slot_src = a.P.f[F_SLOT_SRC];
+  const int64_t nrows = d.R * d.NvS;
+  const int64_t base = k * a.ch + (int64_t)warp * 32 * ppt;
+#pragma unroll
+  for (int j = 0; j < kPairsPerThread; j++) {
+    if (j >= ppt) break;
+    const int64_t p = base + j * 32 + lane;
+    if (p >= d.N) continue;
+    const int e = from_regs ? ev[j] : __ldcs(a.idx + p);
+    const int r = from_regs ? rk[j] : (int)a.rank[p];
+    const int pos = t_base[e] + r;
+    const int kept = t_kept[e];
     int row = -1;
     if (pos < kept) {
-      row = exp_row0[e] + pos;
+      row = t_row0[e] + pos;
     } else {
-      const int o = exp_ostart[e] + (pos - kept);
-      int lo = pbeg[e], hi = pend[e] - 1;  // last piece with ostart <= o
-      if (lo >= 0 && hi >= lo && hi < d.PMAX) {
+      const int o = t_ost[e] + (pos - kept);
+      int lo = t_pb[e], hi = t_pe[e] - 1;  // last piece with ostart <= o
+      if (lo >= 0 && hi >= lo && hi < PM) {
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
-          if (post[mid] <= o) lo = mid; else hi = mid - 1;
+          if (t_post[mid] <= o) lo = mid; else hi = mid - 1;
         }
-        row = piece_grow[lo] + (o - post[lo]);
+        row = t_prow[lo] + (o - t_post[lo]);
       }
     }
     if (row < 0 || row >= nrows) row = -1;  // unreachable for a consistent plan
     slot_of[p] = row;
     if (row >= 0) slot_src[row] = (int32_t)p;
   }
-  // rows that hold no pair: everything after a bad plan, padding when A > 1
+}
+
+__device__ __forceinline__ bool wait_flag(const int32_t *flag, int v, long long limit_ns) {
+  const unsigned long long t0 = now_ns();
+  while (ld_acquire(flag) != v) {
+    if ((long long)(now_ns() - t0) > limit_ns) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  extern __shared__ __align__(16) int smem[];
+  __shared__ int s_epoch, s_state, s_ok;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Dims &d = a.d;
+  const int E = (int)d.E, PM = (int)d.PMAX;
+  int32_t *gen = a.sync + kSyncGen, *done = a.sync + kSyncDone;
+  int32_t *state_w = a.sync + kSyncState, *tables = a.sync + kSyncTables;
+
+  if (tid == 0) s_epoch = (int)((unsigned)*((volatile int32_t *)gen) + kEpochStep);
+  __syncthreads();
+  const int epoch = s_epoch;
+
+  // ================================================================ solver ==
+  if (blockIdx.x == 0) {
+    if (warp == 0) {
+      const bool ok = warp_wait_all(a.arrive, a.nc + a.phantom, epoch, a.wait_ns);
+      bool b = false;
+      for (int64_t c = lane; c < a.nc; c += 32) b |= __ldcg(a.badmark + c) == epoch;
+      b = __any_sync(0xffffffffu, b);
+      if (lane == 0) s_state = (ok ? 0 : kStTimeout) | (b ? kStBad : 0);
+      __threadfence();
+    }
+    __syncthreads();
+    int st = s_state;
+    if (tid == 0) *((volatile int32_t *)gen) = epoch;  // every CTA read it before arriving
+    SolveSmem m = carve(d, smem);
+    if (st == 0) {
+      if (a.nc > a.workers) chunk_bases(a, m.cnt);
+      else column_sums(a.hist, E, a.nc, m.cnt, m.red);
+      st = solve_core(a, m);
+    }
+    if (tid == 0) {
+      if (st & kStTimeout) set_status(a.status, MOONEP_DEV_TIMEOUT);
+      if (st & kStCapacity) set_status(a.status, MOONEP_DEV_CAPACITY);
+      if (st) {
+        int32_t *sc = a.P.f[F_SCALARS];
+        for (int i = 0; i < 8; i++) sc[i] = 0;
+        sc[S_BAD] = st;
+      }
+      *state_w = st;
+      __threadfence();
+      st_release(done, epoch);
+    }
+    if (st == 0) solve_outputs(a, m);
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release(tables, epoch);
+    }
+    return;
+  }
+
+  // =============================================================== workers ==
+  const int wk = blockIdx.x - 1, W = a.workers;
+  const bool single = a.nc <= W;  // at most one chunk per worker: ids and ranks stay in registers
+  int ev[kPairsPerThread], rk[kPairsPerThread];
+  for (int64_t k = wk; k < a.nc; k += W) {
+    const bool bad = __syncthreads_or(count_chunk(a, k, smem, ev, rk));
+    if (!single) {
+      const int64_t base = k * a.ch + (int64_t)warp * 32 * a.ppt;
+#pragma unroll
+      for (int j = 0; j < kPairsPerThread; j++)
+        if (j < a.ppt && ev[j] >= 0) a.rank[base + j * 32 + lane] = (uint16_t)rk[j];
+      __syncthreads();
+    }
+    if (tid == 0) {
+      if (bad) set_status(a.status, MOONEP_DEV_BAD_EXPERT_ID);
+      a.badmark[k] = bad ? epoch : ~epoch;
+      __threadfence();
+      st_release(a.arrive + k, epoch);
+    }
+  }
+  int *tb = smem;  // placement tables, see place_chunk
+  // base offsets of my chunk: sums of the histograms of the chunks before it
+  // (overlaps the solve; with several chunks per worker the solver writes them)
+  bool ok = true;
+  if (single && wk < a.nc) {
+    if (warp == 0) {
+      const bool w = warp_wait_all(a.arrive, wk, epoch, a.wait_ns);
+      if (lane == 0) s_ok = w;
+    }
+    __syncthreads();
+    ok = s_ok;
+    int *red = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(tb + 6 * E + 2 * PM) + 15) &
+                                       ~uintptr_t(15));
+    if (ok) column_sums(a.hist, E, wk, tb, red);
+  }
+  if (tid == 0) {
+    const bool w = wait_flag(done, epoch, a.wait_ns);
+    s_state = w ? __ldcg(state_w) : kStTimeout;
+    if (!w || !ok) set_status(a.status, MOONEP_DEV_TIMEOUT);
+  }
+  __syncthreads();
+  const bool invalid = s_state != 0 || !ok;
+
+  if (!invalid) {
+    for (int e = tid; e < E; e += kPlanThreads) {
+      tb[E + e] = __ldcg(a.exp_kept + e);
+      tb[2 * E + e] = __ldcg(a.exp_row0 + e);
+      tb[3 * E + e] = __ldcg(a.exp_ostart + e);
+      tb[4 * E + e] = __ldcg(a.P.f[F_EXP_PIECE_BEGIN] + e);
+      tb[5 * E + e] = __ldcg(a.P.f[F_EXP_PIECE_END] + e);
+    }
+    for (int i = tid; i < PM; i += kPlanThreads) {
+      tb[6 * E + i] = __ldcg(a.P.f[F_PIECE_OSTART] + i);
+      tb[6 * E + PM + i] = __ldcg(a.piece_grow + i);
+    }
+    __syncthreads();
+    for (int64_t k = wk; k < a.nc; k += W) {
+      if (!single) {
+        for (int e = tid; e < E; e += kPlanThreads) tb[e] = __ldcg(a.hist + k * E + e);
+        __syncthreads();
+      }
+      place_chunk(a, k, tb, single, ev, rk);
+      if (!single) __syncthreads();
+    }
+  } else {
+    int32_t *slot_of = a.P.f[F_SLOT_OF];
+    for (int64_t k = wk; k < a.nc; k += W)
+      for (int64_t p = k * a.ch + tid; p < (k + 1) * a.ch && p < d.N; p += kPlanThreads) slot_of[p] = -1;
+  }
+
+  // rows that hold no pair: everything after an invalid plan, padding when A > 1
   if (invalid || d.A > 1) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nrows; q += stride) {
+    if (!invalid) {
+      if (tid == 0) s_ok = wait_flag(tables, epoch, a.wait_ns);
+      __syncthreads();
+      if (!s_ok) {
+        if (tid == 0) set_status(a.status, MOONEP_DEV_TIMEOUT);
+        return;
+      }
+    }
+    const int64_t nrows = d.R * d.NvS;
+    const int64_t stride = (int64_t)W * blockDim.x;
+    int32_t *slot_src = a.P.f[F_SLOT_SRC];
+    for (int64_t q = (int64_t)wk * blockDim.x + tid; q < nrows; q += stride) {
       if (invalid) {
         slot_src[q] = -1;
         continue;
       }
       const int h = (int)(q / d.NvS), row = (int)(q % d.NvS);
-      const int nseg = P.f[F_N_SEG][h];
-      const int32_t *st = P.f[F_SEG_START] + (int64_t)h * E;
-      const int32_t *ln = P.f[F_SEG_LEN] + (int64_t)h * E;
-      // last segment with start <= row
-      int lo = 0, hi = nseg - 1;
+      const int nseg = __ldcg(a.P.f[F_N_SEG] + h);
+      const int32_t *st = a.P.f[F_SEG_START] + (int64_t)h * E;
+      const int32_t *ln = a.P.f[F_SEG_LEN] + (int64_t)h * E;
+      int lo = 0, hi = nseg - 1;  // last segment with start <= row
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (st[mid] <= row) lo = mid; else hi = mid - 1;
+        if (__ldcg(st + mid) <= row) lo = mid; else hi = mid - 1;
       }
-      // among segments sharing that start (empty ones), the non-empty one is last
-      const bool inside = nseg > 0 && st[lo] <= row && row < st[lo] + ln[lo];
+      const bool inside = nseg > 0 && __ldcg(st + lo) <= row && row < __ldcg(st + lo) + __ldcg(ln + lo);
       if (!inside) slot_src[q] = -1;
     }
   }
 }
 
-size_t solve_smem_bytes(const Dims &d) {
-  const size_t hist_phase = size_t(kPlanWarps) * d.E * sizeof(int);
-  const size_t solve_phase = (9 * d.E + 16 * d.R + 6 * d.PMAX + 40) * sizeof(int);
-  return hist_phase > solve_phase ? hist_phase : solve_phase;
+size_t plan_smem_bytes(const Dims &d) {
+  const size_t worker = std::max<size_t>(size_t(kPlanWarps) * d.E,
+                                         6 * d.E + 2 * d.PMAX + 4 + 4 * kPlanThreads);
+  const size_t solver = solve_smem_ints(d);
+  return std::max(worker, solver) * sizeof(int) + 16;
 }
 
 }  // namespace
@@ -600,35 +840,72 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   if (!plan_arena || !workspace || !dev_status || (d.N > 0 && !topk_idx))
     return MOONEP_ERR_INVALID_ARG;
   if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
-  cudaStream_t st = to_cuda(stream);
-  PlanPtrs P = plan_ptrs(d, plan_arena);
+  const size_t smem = plan_smem_bytes(d);
+  if (smem > 227 * 1024) return MOONEP_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return MOONEP_ERR_CUDA;
+  // co-resident CTAs: a cooperative launch guarantees they run at the same time
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kPlanThreads, smem) !=
+          cudaSuccess)
+    return MOONEP_ERR_CUDA;
+  const int64_t coresident = (int64_t)sms * per_sm;
+  if (coresident < 2) return MOONEP_ERR_UNSUPPORTED;
+
+  PlanArgs a;
+  a.d = d;
+  // chunk size: spread the pairs over every co-resident worker, 512..8192 pairs
+  const int64_t wmax = coresident - 1;
+  int64_t ppt = (d.N + wmax * kPlanThreads - 1) / (wmax * kPlanThreads);
+  ppt = ppt < 1 ? 1 : (ppt > kPairsPerThread ? kPairsPerThread : ppt);
+  a.ppt = (int)ppt;
+  a.ch = ppt * kPlanThreads;
+  a.nc = d.N > 0 ? (d.N + a.ch - 1) / a.ch : 1;
+  a.workers = (int)(a.nc < wmax ? a.nc : wmax);
+  if (a.nc > d.NCMAX) return MOONEP_ERR_UNSUPPORTED;  // cannot happen: chunks >= 512 pairs
+  a.idx = topk_idx;
+  a.P = plan_ptrs(d, plan_arena);
   WsLayout wl(d);
   char *ws = static_cast<char *>(workspace);
-  int32_t *wsflags = reinterpret_cast<int32_t *>(ws + wl.off[W_COUNTER]);
-  int32_t *hist = reinterpret_cast<int32_t *>(ws + wl.off[W_HIST]);
-  uint16_t *rank = reinterpret_cast<uint16_t *>(ws + wl.off[W_RANK]);
-  int32_t *kept = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_KEPT]);
-  int32_t *row0 = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_ROW0]);
-  int32_t *ostart = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_OSTART]);
-  int32_t *grow = reinterpret_cast<int32_t *>(ws + wl.off[W_PIECE_GROW]);
+  a.sync = reinterpret_cast<int32_t *>(ws + wl.off[W_SYNC]);
+  a.arrive = reinterpret_cast<int32_t *>(ws + wl.off[W_ARRIVE]);
+  a.badmark = reinterpret_cast<int32_t *>(ws + wl.off[W_BADMARK]);
+  a.hist = reinterpret_cast<int32_t *>(ws + wl.off[W_HIST]);
+  a.rank = reinterpret_cast<uint16_t *>(ws + wl.off[W_RANK]);
+  a.exp_kept = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_KEPT]);
+  a.exp_row0 = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_ROW0]);
+  a.exp_ostart = reinterpret_cast<int32_t *>(ws + wl.off[W_EXP_OSTART]);
+  a.piece_grow = reinterpret_cast<int32_t *>(ws + wl.off[W_PIECE_GROW]);
+  a.status = dev_status;
+  a.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  a.phantom = g_phantom_arrivals.load(std::memory_order_relaxed);
 
-  if (cudaMemsetAsync(wsflags, 0, 8 * sizeof(int32_t), st) != cudaSuccess) return MOONEP_ERR_CUDA;
-  const size_t smem = solve_smem_bytes(d);
-  if (smem > 48 * 1024) {
-    if (smem > 227 * 1024) return MOONEP_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(plan_hist_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return MOONEP_ERR_CUDA;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)(a.workers + 1));
+  lc.blockDim = dim3(kPlanThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = to_cuda(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, plan_kernel, a) != cudaSuccess) {
+    cudaGetLastError();
+    return MOONEP_ERR_CUDA;
   }
-  plan_hist_solve_kernel<<<(unsigned)d.NC, kPlanThreads, smem, st>>>(
-      d, topk_idx, P, wsflags, hist, rank, kept, row0, ostart, grow, dev_status);
-  if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
-  int64_t blocks = (d.N + kPlacePairsPerBlock - 1) / kPlacePairsPerBlock;
-  if (d.A > 1 && blocks < 148) blocks = 148;
-  if (blocks < 1) blocks = 1;
-  plan_place_kernel<<<(unsigned)blocks, kPlaceThreads, 0, st>>>(d, topk_idx, P, wsflags, hist, rank,
-                                                                 kept, row0, ostart, grow);
-  if (cudaGetLastError() != cudaSuccess) return MOONEP_ERR_CUDA;
+  return MOONEP_OK;
+}
+
+extern "C" moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals) {
+  if (limit_ns < 0 || phantom_arrivals < 0 || phantom_arrivals > kSyncMaxPhantom)
+    return MOONEP_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(limit_ns);
+  g_phantom_arrivals.store(phantom_arrivals);
   return MOONEP_OK;
 }
 
@@ -658,8 +935,8 @@ extern "C" moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const 
       return MOONEP_ERR_CUDA;
     g_plan_scratch_addr[dev].store(scratch, std::memory_order_release);
   }
-  // the ordinary plan with the static array as its workspace (it resets the
-  // arrival counter and flags itself; every other scratch word is written
-  // before it is read)
+  // the ordinary plan with the static array as its workspace: every scratch
+  // word it reads is written earlier in the same call, and its arrival flags
+  // are tagged with a per-launch epoch, so nothing needs clearing
   return moonep_plan(cfg, topk_idx, plan_arena, scratch, dev_status, stream);
 }
