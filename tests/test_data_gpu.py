@@ -227,3 +227,19 @@ def test_reduce_grad_without_budget_is_a_no_op():
     home = integer_bf16((16, 16), seed=9)
     got = _reduce(cfg, arena, np.zeros((4, 0, 16), np.uint16), home, 16)
     assert np.array_equal(got, home)
+
+
+def test_reduce_grad_expert_with_many_pieces():
+    """All tokens on expert 0: its overflow becomes one piece on each of the 7 other ranks."""
+    R, E, K, S, B, P = 8, 16, 1, 64, 2, 520
+    cfg, ocfg = configs(R, E, K, S, H=8, budget=B)
+    idx = np.zeros((R, S, K), np.int32)
+    ost, ot = oracle.plan(ocfg, idx)
+    gst, arena, gv, _ = gpu_plan(cfg, idx)
+    assert int(ot["n_piece"][0]) == R - 1
+    rep = normal_bf16((R, B, P), seed=7, stream=11)
+    home = normal_bf16((E, P), seed=7, stream=12)
+    got = _reduce(cfg, arena, rep, home, P)
+    ref = oracle.reduce_grad(ocfg, ot, rep, home)
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999

@@ -403,9 +403,11 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
 }
 
 // ----------------------------------------------------------- reduce_grad ---
-// Work units: (replicated expert, column vector).  Each unit reads the home
-// vector, adds the expert's local replica vectors in plan order, writes home.
-template <int U>
+// Work units: (replicated expert, warp-chunk of 32*U column vectors).  Each
+// unit reads the home vectors, then the expert's pieces in plan order in groups
+// of G: the group's local replica vectors are all loaded before they are added,
+// so a warp keeps (G + 1) * U loads in flight; adds stay in ascending piece order.
+template <int U, int G>
 __global__ void __launch_bounds__(kThreads)
 reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
                        const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
@@ -430,13 +432,12 @@ reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__
       if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
       continue;
     }
-    float acc[U][8];
     uint4 *hrow = home + (int64_t)e * nvec;
+    float acc[U][8];
 #pragma unroll
     for (int u = 0; u < U; u++) {
       const int64_t v = v0 + u * 32 + lane;
-      uint4 q = make_uint4(0, 0, 0, 0);
-      if (v < nvec) q = hrow[v];
+      const uint4 q = v < nvec ? hrow[v] : make_uint4(0, 0, 0, 0);
       const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int i = 0; i < 4; i++) {
@@ -444,20 +445,32 @@ reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__
         acc[u][2 * i + 1] = bf16_hi(wd[i]);
       }
     }
-    for (int pc = b; pc < en; pc++) {
-      const int ws = pwslot[pc], rk = prank[pc];
-      if (ws < 0) continue;
-      if (ws >= B || rk < 0 || rk >= R) {
-        if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
-        continue;
-      }
-      const uint4 *rrow = rep + ((int64_t)rk * B + ws) * nvec;
+    for (int pc0 = b; pc0 < en; pc0 += G) {
+      uint4 q[G][U];
+      bool use[G];
 #pragma unroll
-      for (int u = 0; u < U; u++) {
-        const int64_t v = v0 + u * 32 + lane;
-        if (v < nvec) {
-          const uint4 q = __ldcs(rrow + v);
-          const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+      for (int g = 0; g < G; g++) {
+        const int pc = pc0 + g;
+        const int ws = pc < en ? pwslot[pc] : -1;
+        const int rk = pc < en ? prank[pc] : -1;
+        use[g] = ws >= 0;
+        if (use[g] && (ws >= B || rk < 0 || rk >= R)) {
+          if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+          use[g] = false;
+        }
+        const uint4 *rrow = rep + ((int64_t)(use[g] ? rk : 0) * B + (use[g] ? ws : 0)) * nvec;
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int64_t v = v0 + u * 32 + lane;
+          q[g][u] = (use[g] && v < nvec) ? __ldcs(rrow + v) : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; g++) {
+        if (!use[g]) continue;
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const uint32_t wd[4] = {q[g][u].x, q[g][u].y, q[g][u].z, q[g][u].w};
 #pragma unroll
           for (int i = 0; i < 4; i++) {
             acc[u][2 * i] = __fadd_rn(acc[u][2 * i], bf16_lo(wd[i]));
@@ -636,7 +649,7 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
   cudaStream_t st = to_cuda(stream);
   const unsigned grid = (unsigned)num_sms() * 8;
   if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
-    reduce_grad_vec_kernel<4><<<grid, kThreads, 0, st>>>(
+    reduce_grad_vec_kernel<4, 4><<<grid, kThreads, 0, st>>>(
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(rep_grads),
         reinterpret_cast<uint4 *>(home_grads), P_elems / 8, (int)d.R, (int)d.E, (int)d.B,
