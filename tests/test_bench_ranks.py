@@ -1,0 +1,74 @@
+"""Multi-process host logic of bench.py, on CPU with gloo (world size 2).
+
+With N GPUs every rank runs an independent replica of the layer (weak scaling,
+no data-path collective); the only communication is the max over ranks of the
+timings, from which rank 0 reports bytes of all ranks / the slowest time.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        mine = [1.5 * rank + 1.0, 10.0 - rank, 3.0]
+        got = bench.max_over_ranks(dist, mine, "cpu")
+        value = bench.whole_job_gbs(4e9, world, got[1])
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"max": got, "value": value}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value(tmp_path):
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mp.start_processes(_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(2)]
+    for r in res:
+        assert r["max"] == [2.5, 10.0, 3.0]
+        # 2 ranks x 4 GB each over the slowest rank's 10 ms
+        assert r["value"] == pytest.approx(8e9 / 10e-3 / 1e9)
+
+
+def test_single_process_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(None, [1.0, 2.0], "cpu") == [1.0, 2.0]
+    assert bench.whole_job_gbs(6.5e9, 1, 1.0) == pytest.approx(6500.0)
+    b = bench.algorithmic_bytes(8, 4096, 8, 7168)
+    assert b["dispatch"] == 4228907008 and b["combine"] == 4229955584
+
+
+@pytest.mark.parametrize("rank", [0, 1])
+def test_reference_arm_runs_on_rank_zero_only(rank):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "ep8_e32_k4_s256_h512", "--steps", "3", "--warmup", "1",
+                        "--reference-budget-s", "5"], capture_output=True, text=True, env=env,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    if rank == 0:
+        assert len(lines) == 1
+        d = json.loads(lines[0])
+        assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+        assert d["cpu_baseline"]["kind"] == "oracle" and d["n_gpus"] == 2
+        assert d["e2e"]["h2d_bytes_per_step"] == 0
+    else:
+        assert lines == []

@@ -1,0 +1,129 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times.
+
+The oracle computes sampled outputs one by one from host inputs (it never reads
+a buffer the GPU produced): for the identity expert the K rows a token gathers
+are its own row of x.  Whole-buffer properties are checked on the device with
+the oracle's plan (every valid row of the dispatch buffer equals its source
+token's row; padding rows untouched).
+Tolerance: bit-exact for the plan and dispatched rows; 1e-3 norm-relative for
+combine, combine-backward and reduce_grad (fp32 accumulation).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from moonep_inputs import (WORKLOADS, bf16_bits_to_f32, make_dout, make_gates, make_routing,
+                           make_x, row_pool)
+from tests.gpu_util import compare_plans, rel_err, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+N_SAMPLE_TOKENS = 384
+N_SAMPLE_COLS = 2048
+
+
+@pytest.mark.parametrize("name,mv", [("ep8_e256_k8_s4096_h7168", 0.2),
+                                     ("ep8_e384_k8_s8192_h7168_bwd", 20.0),
+                                     ("ep64_e256_k8_s128_h7168_decode", 20.0)])
+def test_full_size_layer(name, mv):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    w = WORKLOADS[name]
+    R, E, K, S, H, B = w.R, w.E, w.K, w.S, w.H, w.budget
+    T = R * S
+    train = w.mode == 0
+    cfg = me.Config.of(w)
+    ocfg = oracle.Config.of(w)
+    idx, _, _ = make_routing(R, E, K, S, mv, seed=0)
+    gates = make_gates(R, S, K, seed=0).reshape(T, K)
+    x = make_x(R, S, H, seed=0).reshape(T, H)
+    NvS = me.moonep_nvs(cfg)
+    dev = torch.device("cuda")
+    POISON = -63  # 0xFFC1 as int16
+
+    # ---- plan (bit-exact, every table)
+    ost, ot = oracle.plan(ocfg, idx)
+    arena, ws, status = me.alloc_plan(cfg)
+    idx_d = to_dev(idx.ravel().astype(np.int32))
+    me.moonep_plan(cfg, idx_d, arena, ws, status)
+    torch.cuda.synchronize()
+    gv = {k: (to_np(v) if not isinstance(v, int) else v)
+          for k, v in me.moonep_plan_view(cfg, arena).items()}
+    compare_plans(cfg, ost, ot, int(status.item()), gv)
+
+    # ---- dispatch
+    x_d = to_dev(x)
+    recv = torch.full((R * NvS, H), POISON, dtype=torch.int16, device=dev)
+    me.moonep_dispatch(cfg, arena, x_d, recv, status)
+    torch.cuda.synchronize()
+    src = torch.from_numpy(ot["slot_src"].astype(np.int64)).to(dev)
+    valid = src >= 0
+    # property over the whole buffer: valid rows are their source token's row, padding untouched
+    assert torch.equal(recv[valid], x_d[src[valid] // K])
+    assert bool((recv[~valid] == POISON).all())
+    rng = np.random.default_rng(1)
+    rows = rng.choice(np.nonzero(ot["slot_src"] >= 0)[0], size=min(2048, T * K), replace=False)
+    got_rows = to_np(recv[torch.from_numpy(rows).to(dev)])
+    assert np.array_equal(got_rows, x[ot["slot_src"][rows] // K])
+
+    # ---- combine (identity expert: y = the dispatch buffer)
+    g_d = to_dev(gates.ravel())
+    out = torch.empty((T, H), dtype=torch.int16, device=dev)
+    me.moonep_combine(cfg, arena, recv, g_d, out, status)
+    torch.cuda.synchronize()
+    toks = np.sort(rng.choice(T, size=min(N_SAMPLE_TOKENS, T), replace=False))
+    n = len(toks)
+    c1 = oracle.Config(R=1, E=E, K=K, S=n, H=H, budget=B, mode=w.mode)
+    y_rows = np.repeat(x[toks], K, axis=0)                 # row k of token t is x[t]
+    compact = np.arange(n * K, dtype=np.int32)
+    ref_out = oracle.combine(c1, compact, y_rows, gates[toks])
+    got_out = to_np(out[torch.from_numpy(toks).to(dev)])
+    assert rel_err(bf16_bits_to_f32(got_out), bf16_bits_to_f32(ref_out)) <= TOL
+    assert (got_out == ref_out).mean() >= 0.999
+    del out
+    torch.cuda.synchronize()
+
+    if not train:
+        assert int(status.item()) == 0
+        return
+
+    # ---- combine-backward
+    dout = make_dout(R, S, H, seed=0).reshape(T, H)
+    dout_d = to_dev(dout)
+    dy = torch.full((R * NvS, H), POISON, dtype=torch.int16, device=dev)
+    dg = torch.empty(T * K, dtype=torch.float32, device=dev)
+    me.moonep_combine_backward(cfg, arena, dout_d, recv, g_d, dy, dg, status)
+    torch.cuda.synchronize()
+    ref_dy, ref_dg = oracle.combine_backward(c1, compact, dout[toks], y_rows, gates[toks])
+    so = torch.from_numpy(ot["slot_of"].reshape(T, K)[toks].ravel().astype(np.int64)).to(dev)
+    got_dy = to_np(dy[so]).reshape(n, K, H)
+    assert rel_err(bf16_bits_to_f32(got_dy), bf16_bits_to_f32(ref_dy)) <= TOL
+    assert (got_dy == ref_dy).mean() >= 0.999
+    got_dg = to_np(dg).reshape(T, K)[toks]
+    assert rel_err(got_dg, ref_dg) <= TOL
+    assert bool((dy[~valid] == POISON).all())
+    del dy, dg, recv, dout_d, x_d
+    torch.cuda.empty_cache()
+
+    # ---- reduce_grad on [2048 x H] expert gradients built from a pool of rows
+    P = w.P
+    pool = row_pool(12, P, seed=3)                          # 12 bf16 rows of P elements
+    rep_map = (np.arange(R * B) * 7 + 3) % 12               # replica slot -> pool row
+    home_map = (np.arange(E) * 5 + 1) % 12                  # expert -> pool row
+    pool_d = to_dev(pool)
+    rep = pool_d[torch.from_numpy(rep_map).to(dev)]         # [R*B, P] on the device
+    home = pool_d[torch.from_numpy(home_map).to(dev)]       # [E, P]
+    me.moonep_reduce_grad(cfg, arena, rep, home, P, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    cols = np.sort(rng.choice(P, size=N_SAMPLE_COLS, replace=False))
+    rep_cols = pool[rep_map][:, cols].reshape(R, B, len(cols))
+    home_cols = pool[home_map][:, cols]
+    ref_home = oracle.reduce_grad(ocfg, ot, rep_cols, home_cols)
+    got_home = to_np(home[:, torch.from_numpy(cols).to(dev)])
+    assert rel_err(bf16_bits_to_f32(got_home), bf16_bits_to_f32(ref_home)) <= TOL
+    assert (got_home == ref_home).mean() >= 0.999
+    touched = np.zeros(E, bool)
+    touched[ot["piece_expert"][ot["piece_wslot"] >= 0]] = True
+    assert touched.any()
+    assert np.array_equal(got_home[~touched], home_cols[~touched])  # untouched experts unchanged
