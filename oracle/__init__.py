@@ -31,6 +31,7 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
 from __future__ import annotations
 
 import ctypes
+import os
 from typing import Dict, Optional, Tuple
 
 import numpy as np
@@ -79,7 +80,9 @@ _lib = None
 def _L():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # MOONEP_ORACLE_LIB: a deliberately broken oracle build, used only by the test that
+        # checks the pins fail against planted mistakes
+        lib = ctypes.CDLL(os.environ.get("MOONEP_ORACLE_LIB") or build())
         vp = ctypes.c_void_p
         cp = ctypes.POINTER(Config)
         lib.orc_nvs.argtypes = [cp]

@@ -1,0 +1,55 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a scratch copy of oracle/moonep_oracle.c
+(wrong keep/overflow cut, wrong receiver order, wrong layout, wrong weight
+slot, a dropped term, a missing gate, a skipped replica, ignored alignment,
+truncating instead of rounding, reversed per-expert order, a half dot
+product), builds it with gcc, and runs the pin tests against it: at least one
+pin must fail.  Everything runs on the CPU.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "moonep_oracle.c")
+
+MUTANTS = {
+    "keep_tail_not_head": ("if (t < SK) {", "if (t >= out->rank_load[h] - SK) {"),
+    "receivers_descending": ("for (d = 0; d < R; d++) {\n    int64_t need",
+                             "for (d = R - 1; d >= 0; d--) {\n    int64_t need"),
+    "native_segments_missing": ("for (e = d * L; e < (d + 1) * L; e++) {\n      int64_t idx = d * E + nseg;",
+                                "for (e = d * L; e < (d + 1) * L && 0; e++) {\n      int64_t idx = d * E + nseg;"),
+    "weight_slot_off_by_one": ("out->piece_wslot[n_piece] = (int32_t)j;",
+                               "out->piece_wslot[n_piece] = (int32_t)(j + 1 < B ? j + 1 : j);"),
+    "combine_drops_last_k": ("for (int64_t k = 0; k < K; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc",
+                             "for (int64_t k = 0; k < K - 1; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc"),
+    "backward_without_gate": ("float prod = w * g;", "float prod = g;"),
+    "reduce_skips_first_piece": ("acc = acc + orc_bf16_to_f32(rep[slot * P + q]);",
+                                 "if (i > 0) acc = acc + orc_bf16_to_f32(rep[slot * P + q]);"),
+    "alignment_ignored": ("cursor += roundup64(kept[e], A);", "cursor += kept[e];"),
+    "truncate_not_round": ("u += 0x7FFFu + lsb;", "u += 0;"),
+    "expert_list_reversed": ("list[list_begin[e] + fill[e]] = p;",
+                             "list[list_begin[e + 1] - 1 - fill[e]] = p;"),
+    "half_dot_product": ("dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);",
+                         "if (h % 2 == 0) dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found once: {name}"
+    mut_c = tmp_path / "mutant.c"
+    mut_c.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-w", "-o", str(lib), str(mut_c), "-lm"])
+    env = dict(os.environ, MOONEP_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin caught the mutant '{name}':\n{r.stdout[-1500:]}"
