@@ -2,8 +2,9 @@
 """Benchmark of the MoonEP balanced expert-parallel hot path on B200.
 
 One step = one MoE layer's pass of the whole hot path over a fresh batch of
-router output: plan -> zero-copy dispatch -> identity expert -> combine, and in
-training mode combine-backward -> reduce_grad of replica expert gradients.
+router output: plan -> (training: prefetch of replica weights) -> zero-copy
+dispatch -> identity expert -> combine, and in training mode combine-backward ->
+dispatch-backward -> reduce_grad of replica expert gradients.
 Inputs are synthetic and seeded (Zipf-popular experts, Gumbel-top-k picks,
 softmax gates, N(0,1) bf16 rows; see moonep_inputs).
 
@@ -57,6 +58,8 @@ def algorithmic_bytes(R, S, K, H, n_local=0, n_rep_exp=0, P=0):
         "combine": RSK * H * 2 + T * H * 2 + RSK * 8,
         "combine_bwd": T * H * 2 + 2 * RSK * H * 2 + RSK * 12,
         "reduce_grad": n_local * P * 2 + n_rep_exp * P * 2 * 2,
+        "prefetch": n_rep_exp * P * 2 + n_local * P * 2,  # home weights read once, replicas written
+        "dispatch_bwd": RSK * H * 2 + T * H * 2 + RSK * 4,
     }
 
 
@@ -199,12 +202,16 @@ class Layer:
                 step = 1 << 28
                 for i in range(0, n, step):
                     buf[i:i + step].copy_(torch.randn(min(step, n - i), generator=g, device=device))
+            self.dx = torch.empty(T * H, dtype=torch.int16, device=device)
+            self.weights = torch.empty(E * self.P, dtype=torch.bfloat16, device=device)
+            self.rep_w = torch.empty(R * w.budget * self.P, dtype=torch.bfloat16, device=device)
+            self.weights.copy_(self.home)  # any bf16 values: the copy moves bits
             self.h_out = torch.empty(T * H, dtype=torch.int16).pin_memory() if pin else None
             self.h_dg = torch.empty(T * K, dtype=torch.float32).pin_memory() if pin else None
         else:
             self.P = 0
             self.h_out = torch.empty(T * H, dtype=torch.int16).pin_memory() if pin else None
-        self.launches_per_step = 3 + (2 if self.train else 0)  # the plan is one kernel
+        self.launches_per_step = 3 + (4 if self.train else 0)  # the plan is one kernel
         self.n_local = self.n_rep_exp = 0
         self.e2e_bufs = None
 
@@ -230,14 +237,19 @@ class Layer:
         me, c = self.me, self.cfg
         b = buf or dict(idx=self.idx, gates=self.gates, x=self.x, out=self.out,
                         dout=getattr(self, "dout", None), dg=getattr(self, "dg", None))
-        seq = [("plan", lambda: me.moonep_plan(c, b["idx"], self.arena, self.ws, self.status)),
-               ("dispatch", lambda: me.moonep_dispatch(c, self.arena, b["x"], self.recv, self.status)),
+        seq = [("plan", lambda: me.moonep_plan(c, b["idx"], self.arena, self.ws, self.status))]
+        if self.train:
+            seq += [("prefetch", lambda: me.moonep_prefetch_weight(c, self.arena, self.weights, self.rep_w,
+                                                                   self.P, self.status))]
+        seq += [("dispatch", lambda: me.moonep_dispatch(c, self.arena, b["x"], self.recv, self.status)),
                ("combine", lambda: me.moonep_combine(c, self.arena, self.recv, b["gates"], b["out"],
                                                      self.status))]
         if self.train:
             seq += [("combine_bwd", lambda: me.moonep_combine_backward(
                         c, self.arena, b["dout"], self.recv, b["gates"], self.dy, b["dg"],
                         self.status)),
+                    ("dispatch_bwd", lambda: me.moonep_dispatch_backward(c, self.arena, self.dy, self.dx,
+                                                                         self.status)),
                     ("reduce_grad", lambda: me.moonep_reduce_grad(c, self.arena, self.rep, self.home,
                                                                   self.P, self.status))]
         return seq
@@ -252,8 +264,8 @@ class Layer:
         w = self.w
         b = algorithmic_bytes(w.R, w.S, w.K, w.H, self.n_local, self.n_rep_exp, self.P)
         if not self.train:
-            b.pop("combine_bwd")
-            b.pop("reduce_grad")
+            for k in ("combine_bwd", "reduce_grad", "prefetch", "dispatch_bwd"):
+                b.pop(k)
         return b
 
 
@@ -551,7 +563,8 @@ def main():
                        "R": w.R, "E": w.E, "K": w.K, "S": w.S, "H": w.H, "budget": w.budget,
                        "mode": "train" if w.mode == MODE_TRAIN else "infer",
                        "maxvio": round(layer.maxvio, 4), "zipf_alpha": round(layer.alpha, 4),
-                       "step": "plan+dispatch+combine" + ("+combine_bwd+reduce_grad" if layer.train else ""),
+                       "step": ("plan+prefetch+dispatch+combine+combine_bwd+dispatch_bwd+reduce_grad"
+                                if layer.train else "plan+dispatch+combine"),
                        "grad_elems_per_expert": layer.P,
                        "l2": "inputs larger than L2 (x %.0f MB, dispatch buffer %.0f MB); no flush"
                              % (layer.x.numel() * 2 / 1e6, layer.recv.numel() * 2 / 1e6),

@@ -9,6 +9,8 @@
  *   moonep_combine           gate-weighted gather-sum of expert outputs back to tokens
  *   moonep_combine_backward  gradients of combine w.r.t. expert outputs and gates
  *   moonep_reduce_grad       fold replica-expert gradients into their home experts
+ *   moonep_dispatch_backward gradient of dispatch (sum of a token's K slot gradients)
+ *   moonep_prefetch_weight   copy duplicated experts' weights into replica slots
  *
  * Conventions shared by every call:
  *   - Ownership: the caller allocates and frees every buffer (device memory
@@ -223,6 +225,31 @@ MOONEP_API moonep_status_t moonep_combine_backward(const moonep_config_t *cfg, c
 MOONEP_API moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
                                    const uint16_t *rep_grads, uint16_t *home_grads, int64_t P,
                                    int32_t *dev_status, moonep_stream_t stream);
+
+/* Backward of dispatch (reuses the forward plan, "MoonshotAI/MoonEP 딥다이브" §4
+ * pattern 1): the gradient of each token row is the sum of the gradients of
+ * the K slots it was sent to,
+ *   dx[t] = bf16( sum_{k=0..K-1} d_recv[slot_of[t*K+k]] )
+ * accumulated in fp32 in ascending k, rounded once (nearest-even).
+ * d_recv bf16 [R*NvS, H]; dx bf16 [R*S, H]. */
+MOONEP_API moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
+                                                    const void *plan_arena, const uint16_t *d_recv,
+                                                    uint16_t *dx, int32_t *dev_status,
+                                                    moonep_stream_t stream);
+
+/* Replica weight prefetch ("Moonshot AI Open-Sources MoonEP", S x K paragraph:
+ * duplicated experts are prefetched before computation starts; the
+ * replica-slot paragraph: E/R slots in training, 3-4 in inference with remote
+ * reads past the budget; Buffer.prefetch_weight, "MoonshotAI/MoonEP 딥다이브" §3③):
+ *   rep_weights[d, j, :] = weights[e, :] for every piece of expert e that holds
+ *   local weight slot j on rank d (a bit copy; each home row is read once).
+ * Remote pieces (weight slot -1 in the plan) are not copied: their segments
+ * read weights[e] on the home rank.  weights bf16 [E, W]; rep_weights bf16
+ * [R, budget, W] (slots without a piece are left untouched); W >= 1. */
+MOONEP_API moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
+                                                  const void *plan_arena, const uint16_t *weights,
+                                                  uint16_t *rep_weights, int64_t W,
+                                                  int32_t *dev_status, moonep_stream_t stream);
 
 /* Static description of a status code. */
 MOONEP_API const char *moonep_status_string(moonep_status_t status);

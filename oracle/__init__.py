@@ -27,6 +27,12 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
 * ``reduce_grad`` — with integer-valued bf16 gradients all fp32 sums are
   exact, so home + replicas must equal, bit for bit, the no-replication
   gradient (§4 pattern 3, §8 exercise E).
+* ``dispatch_backward`` — the adjoint of dispatch: with integer-valued data
+  <dispatch(x), dR> = <x, dispatch_backward(dR)> exactly, and
+  dispatch_backward(dispatch(x)) = K*x.
+* ``prefetch_weight`` — every local replica slot holds its expert's weights
+  bit for bit, every other slot is untouched; closed form for all tokens on
+  one expert.
 """
 from __future__ import annotations
 
@@ -97,6 +103,10 @@ def _L():
         lib.orc_combine_backward_tokens.restype = None
         lib.orc_reduce_grad.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
         lib.orc_reduce_grad.restype = None
+        lib.orc_dispatch_backward_tokens.argtypes = [cp, vp, vp, vp, ctypes.c_int64, vp]
+        lib.orc_dispatch_backward_tokens.restype = None
+        lib.orc_prefetch_weight.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
+        lib.orc_prefetch_weight.restype = None
         lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.orc_f32_to_bf16.restype = ctypes.c_uint16
         lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -197,6 +207,31 @@ def reduce_grad(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray, hom
     pw = _c(tables["piece_wslot"], np.int32)
     _L().orc_reduce_grad(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(rep), _p(home), P)
     return home
+
+
+def dispatch_backward(cfg: Config, slot_of: np.ndarray, drecv: np.ndarray,
+                      tokens: Optional[np.ndarray] = None) -> np.ndarray:
+    """bf16 bits [n_tokens, H] of sum_k dRecv[slot_k] (fp32, k order) for the listed tokens."""
+    s = _c(slot_of, np.int32)
+    d = _c(drecv, np.uint16)
+    n = cfg.R * cfg.S if tokens is None else len(tokens)
+    tk = None if tokens is None else _c(tokens, np.int64)
+    out = np.zeros((n, cfg.H), np.uint16)
+    _L().orc_dispatch_backward_tokens(ctypes.byref(cfg), _p(s), _p(d), _p(tk), n, _p(out))
+    return out
+
+
+def prefetch_weight(cfg: Config, tables: Dict[str, np.ndarray], w: np.ndarray,
+                    rep_w: np.ndarray) -> np.ndarray:
+    """Replica weight slots after the prefetch (bf16 bits [R, budget, W]); ``w`` is [E, W]."""
+    rep_w = np.array(rep_w, dtype=np.uint16, copy=True, order="C")
+    ww = _c(w, np.uint16)
+    pe = _c(tables["piece_expert"], np.int32)
+    pr = _c(tables["piece_rank"], np.int32)
+    pw = _c(tables["piece_wslot"], np.int32)
+    _L().orc_prefetch_weight(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(ww), _p(rep_w),
+                             ww.shape[-1])
+    return rep_w
 
 
 def f32_to_bf16(v: float) -> int:

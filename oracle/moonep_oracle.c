@@ -47,6 +47,11 @@
  *              dgate[t,k] = sum_h dOut[t,h] * y[slot_k,h] accumulated in double
  *   reduce_grad home[e] = bf16(float(home[e]) + sum over e's local replica pieces,
  *              in O order (ascending receiver), of float(rep[d][slot]))
+ *   dispatch-bw dx[t] = bf16( sum_k float(dRecv[slot_k]) ), fp32 adds in k order (the
+ *              adjoint of dispatch; the backward pass reuses the forward plan, §4 pattern 1)
+ *   prefetch   rep_w[d][j] = w[e] for every local replica piece (d, j) of expert e
+ *              (the duplicated experts' weights are fetched before compute: news page,
+ *              S x K paragraph; Buffer.prefetch_weight, deep-dive §3③)
  * bf16 rounding is round-to-nearest-even on the fp32 bit pattern.
  */
 #include <math.h>
@@ -380,5 +385,38 @@ void orc_reduce_grad(const orc_config *c, const int32_t *piece_expert, const int
       }
       home[e * P + q] = orc_f32_to_bf16(acc);
     }
+  }
+}
+
+/* ------------------------------------------------------ dispatch-backward --- */
+/* dx[t] = bf16( sum_k float(drecv[slot_of[t,k]]) ), fp32 additions in k order. */
+void orc_dispatch_backward_tokens(const orc_config *c, const int32_t *slot_of,
+                                  const uint16_t *drecv, const int64_t *tokens, int64_t n_tokens,
+                                  uint16_t *dx) {
+  const int64_t K = c->K, H = c->H;
+  for (int64_t n = 0; n < n_tokens; n++) {
+    int64_t t = tokens ? tokens[n] : n;
+    for (int64_t h = 0; h < H; h++) {
+      float acc = 0.0f;
+      for (int64_t k = 0; k < K; k++) {
+        int64_t row = slot_of[t * K + k];
+        acc = acc + orc_bf16_to_f32(drecv[row * H + h]);
+      }
+      dx[n * H + h] = orc_f32_to_bf16(acc);
+    }
+  }
+}
+
+/* --------------------------------------------------------- prefetch_weight --- */
+/* For every piece with a local weight slot: rep_w[rank][slot] = w[expert] (W elements).
+   rep_w is [R, budget, W]; w is [E, W]. */
+void orc_prefetch_weight(const orc_config *c, const int32_t *piece_expert,
+                         const int32_t *piece_rank, const int32_t *piece_wslot, int32_t n_piece,
+                         const uint16_t *w, uint16_t *rep_w, int64_t W) {
+  const int64_t B = c->budget;
+  for (int32_t i = 0; i < n_piece; i++) {
+    if (piece_wslot[i] < 0) continue;
+    int64_t slot = (int64_t)piece_rank[i] * B + piece_wslot[i];
+    for (int64_t q = 0; q < W; q++) rep_w[slot * W + q] = w[(int64_t)piece_expert[i] * W + q];
   }
 }

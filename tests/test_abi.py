@@ -86,6 +86,11 @@ def test_null_and_misaligned_pointers_rejected_on_host():
     assert L.moonep_reduce_grad(cp, base, base, base, 0, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_reduce_grad(cp, base, None, base, 16, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_plan_view(cp, None, ctypes.byref(me.PlanView())) == me.ERR_INVALID_ARG
+    assert L.moonep_dispatch_backward(cp, base, None, base, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_dispatch_backward(cp, base, base, None, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_prefetch_weight(cp, base, None, base, 16, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_prefetch_weight(cp, base, base, None, 16, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_prefetch_weight(cp, base, base, base, 0, base, 0) == me.ERR_INVALID_ARG
 
 
 def test_empty_batch_enqueues_nothing():

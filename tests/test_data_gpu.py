@@ -243,3 +243,64 @@ def test_reduce_grad_expert_with_many_pieces():
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
     assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
     assert (got == ref).mean() >= 0.999
+
+
+def _dispatch_bwd(cfg, arena, drecv_np):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    d = to_dev(drecv_np)
+    dx = torch.empty((cfg.R * cfg.S, cfg.H), dtype=torch.int16, device=d.device)
+    status = torch.zeros(1, dtype=torch.int32, device=d.device)
+    me.moonep_dispatch_backward(cfg, arena, d, dx, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return to_np(dx)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_dispatch_backward_matches_oracle(shape):
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A, seed=10)
+    NvS = int(ot["nvs"][0])
+    drecv = normal_bf16((R * NvS, H), seed=10, stream=13)
+    got = _dispatch_bwd(cfg, arena, drecv)
+    ref = oracle.dispatch_backward(ocfg, ot["slot_of"], drecv)
+    if ref.size == 0:
+        assert got.size == 0
+        return
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999
+
+
+def test_dispatch_backward_is_adjoint_on_gpu():
+    """Integer data: <dispatch(x), dR> == <x, dispatch_backward(dR)> exactly, on the GPU path."""
+    R, E, K, S, H = 8, 32, 4, 64, 64
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, seed=11)
+    NvS = int(ot["nvs"][0])
+    x = integer_bf16((R * S, H), seed=11, bound=4)
+    dR = integer_bf16((R * NvS, H), seed=12, bound=4)
+    recv = _dispatch(cfg, arena, x, NvS)
+    dx = _dispatch_bwd(cfg, arena, dR)
+    valid = ot["slot_src"] >= 0
+    lhs = (bf16_bits_to_f32(recv[valid]).astype(np.int64) *
+           bf16_bits_to_f32(dR[valid]).astype(np.int64)).sum()
+    rhs = (bf16_bits_to_f32(x).astype(np.int64) * bf16_bits_to_f32(dx).astype(np.int64)).sum()
+    assert lhs == rhs
+
+
+@pytest.mark.parametrize("shape", [(8, 32, 4, 256, 4, 4096, 0.2), (8, 64, 8, 64, 8, 1000, 6.0),
+                                   (4, 16, 2, 40, 3, 13, 3.0), (64, 256, 8, 16, 4, 512, 20.0)])
+def test_prefetch_weight_matches_oracle(shape):
+    import torch
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S, B, W, mv = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=mv, seed=13, budget=B, mode=1)
+    w = normal_bf16((E, W), seed=13, stream=14)
+    before = normal_bf16((R, B, W), seed=14, stream=15)
+    rep = to_dev(before)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    me.moonep_prefetch_weight(cfg, arena, to_dev(w), rep, W, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ref = oracle.prefetch_weight(ocfg, ot, w, before)
+    assert np.array_equal(to_np(rep), ref)

@@ -33,6 +33,10 @@ MUTANTS = {
     "truncate_not_round": ("u += 0x7FFFu + lsb;", "u += 0;"),
     "expert_list_reversed": ("list[list_begin[e] + fill[e]] = p;",
                              "list[list_begin[e + 1] - 1 - fill[e]] = p;"),
+    "dispatch_backward_drops_first_k": ("acc = acc + orc_bf16_to_f32(drecv[row * H + h]);",
+                                        "if (k > 0) acc = acc + orc_bf16_to_f32(drecv[row * H + h]);"),
+    "prefetch_wrong_expert": ("rep_w[slot * W + q] = w[(int64_t)piece_expert[i] * W + q];",
+                              "rep_w[slot * W + q] = w[(int64_t)((piece_expert[i] + 1) % c->E) * W + q];"),
     "half_dot_product": ("dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);",
                          "if (h % 2 == 0) dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);"),
 }

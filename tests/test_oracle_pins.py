@@ -546,3 +546,88 @@ def test_reduce_grad_leaves_unreplicated_experts_alone():
         for i in np.nonzero((t["piece_expert"] == e) & (t["piece_wslot"] >= 0))[0]:
             want += rf[t["piece_rank"][i], t["piece_wslot"][i]]
         assert np.array_equal(bf16_bits_to_f32(new[e]).astype(np.int64), want)
+
+
+# ------------------------------------------------------- dispatch-backward ---
+
+
+@pytest.mark.parametrize("case", [(8, 32, 4, 48, 24, 3.0), (3, 9, 3, 17, 8, 1.0),
+                                  (4, 16, 8, 10, 16, 5.0)])
+def test_dispatch_backward_is_the_adjoint_of_dispatch(case):
+    """<dispatch(x), dR> = <x, dispatch_backward(dR)> with integers (all sums exact)."""
+    R, E, K, S, H, mv = case
+    idx, _, _ = make_routing(R, E, K, S, mv, seed=12)
+    c = cfg(R, E, K, S, H=H)
+    st, t = oracle.plan(c, idx)
+    NvS = int(t["nvs"][0])
+    x = integer_bf16((R * S, H), seed=12, bound=4)
+    dR = integer_bf16((R * NvS, H), seed=13, bound=4)
+    recv = oracle.dispatch(c, t["slot_of"], x)
+    dx = oracle.dispatch_backward(c, t["slot_of"], dR)
+    valid = t["slot_src"] >= 0
+    lhs = (bf16_bits_to_f32(recv[valid]).astype(np.int64) *
+           bf16_bits_to_f32(dR[valid]).astype(np.int64)).sum()
+    rhs = (bf16_bits_to_f32(x).astype(np.int64) * bf16_bits_to_f32(dx).astype(np.int64)).sum()
+    assert lhs == rhs
+    # per element: dx[t] is the sum of the K rows that token t was sent to
+    ref = bf16_bits_to_f32(dR).astype(np.int64)[t["slot_of"]].reshape(R * S, K, H).sum(1)
+    assert np.array_equal(bf16_bits_to_f32(dx).astype(np.int64), ref)
+
+
+def test_dispatch_backward_of_dispatch_is_k_times_x():
+    R, E, K, S, H = 4, 16, 4, 20, 32
+    idx, _, _ = make_routing(R, E, K, S, 2.0, seed=14)
+    c = cfg(R, E, K, S, H=H)
+    st, t = oracle.plan(c, idx)
+    x = integer_bf16((R * S, H), seed=14, bound=32)
+    dx = oracle.dispatch_backward(c, t["slot_of"], oracle.dispatch(c, t["slot_of"], x))
+    assert np.array_equal(bf16_bits_to_f32(dx), K * bf16_bits_to_f32(x))
+
+
+def test_dispatch_backward_rounding_bound():
+    R, E, K, S, H = 4, 16, 8, 12, 40
+    idx, _, _ = make_routing(R, E, K, S, 3.0, seed=15)
+    c = cfg(R, E, K, S, H=H)
+    st, t = oracle.plan(c, idx)
+    NvS = int(t["nvs"][0])
+    dR = normal_bf16((R * NvS, H), seed=15, stream=21)
+    dx = oracle.dispatch_backward(c, t["slot_of"], dR)
+    terms = bf16_bits_to_f32(dR).astype(np.float64)[t["slot_of"]].reshape(R * S, K, H)
+    exact = terms.sum(1)
+    bound = _bf16_half_ulp(exact) * (1 + 2 ** -7) + K * 2.0 ** -23 * np.abs(terms).sum(1)
+    assert (np.abs(bf16_bits_to_f32(dx) - exact) <= bound).all()
+
+
+# --------------------------------------------------------- prefetch_weight ---
+
+
+@pytest.mark.parametrize("case", [(8, 32, 4, 64, 4, 6.0), (4, 16, 2, 40, 1, 4.0)])
+def test_prefetch_copies_home_weights_into_local_slots(case):
+    R, E, K, S, B, mv = case
+    idx, _, _ = make_routing(R, E, K, S, mv, seed=16)
+    c = cfg(R, E, K, S, budget=B, mode=1)
+    st, t = oracle.plan(c, idx)
+    W = 20
+    w = normal_bf16((E, W), seed=16, stream=22)
+    before = normal_bf16((R, B, W), seed=17, stream=23)
+    after = oracle.prefetch_weight(c, t, w, before)
+    filled = np.zeros((R, B), bool)
+    for d in range(R):
+        for j in range(B):
+            e = t["rep_expert"][d * B + j]
+            if e >= 0:
+                assert np.array_equal(after[d, j], w[e])
+                filled[d, j] = True
+    assert np.array_equal(after[~filled], before[~filled])
+    assert filled.sum() == int((t["piece_wslot"] >= 0).sum())
+
+
+def test_prefetch_all_tokens_on_one_expert():
+    """Expert 0's overflow lands on every other rank, each holding its weights in slot 0."""
+    R, S = 4, 6
+    c = cfg(R, R, 1, S, budget=2, mode=1)
+    st, t = oracle.plan(c, np.zeros((R, S, 1), np.int32))
+    w = normal_bf16((R, 8), seed=18, stream=24)
+    after = oracle.prefetch_weight(c, t, w, np.zeros((R, 2, 8), np.uint16))
+    assert np.array_equal(after[1:, 0], np.broadcast_to(w[0], (R - 1, 8)))
+    assert not after[0].any() and not after[1:, 1].any()

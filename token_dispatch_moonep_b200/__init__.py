@@ -16,6 +16,8 @@ The functions keep the C names::
     moonep_combine(cfg, plan_arena, y, gates, out, dev_status, stream=None)
     moonep_combine_backward(cfg, plan_arena, dout, y, gates, dy, dgates, dev_status, stream=None)
     moonep_reduce_grad(cfg, plan_arena, rep_grads, home_grads, P, dev_status, stream=None)
+    moonep_dispatch_backward(cfg, plan_arena, d_recv, dx, dev_status, stream=None)
+    moonep_prefetch_weight(cfg, plan_arena, weights, rep_weights, W, dev_status, stream=None)
 
 Tensor arguments are device tensors (bf16 tensors may be ``torch.bfloat16``
 or ``int16``/``uint16`` views); raw integer device addresses are accepted too.
@@ -127,6 +129,10 @@ _lib.moonep_combine_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
 _lib.moonep_combine_backward.restype = _ST
 _lib.moonep_reduce_grad.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
 _lib.moonep_reduce_grad.restype = _ST
+_lib.moonep_dispatch_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
+_lib.moonep_dispatch_backward.restype = _ST
+_lib.moonep_prefetch_weight.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
+_lib.moonep_prefetch_weight.restype = _ST
 _lib.moonep_status_string.argtypes = [_ST]
 _lib.moonep_status_string.restype = ctypes.c_char_p
 
@@ -249,6 +255,19 @@ def moonep_reduce_grad(cfg: Config, plan_arena, rep_grads, home_grads, P: int, d
                        stream=None) -> None:
     _check("moonep_reduce_grad", _lib.moonep_reduce_grad(
         ctypes.byref(cfg), _ptr(plan_arena), _ptr(rep_grads), _ptr(home_grads), int(P),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moonep_dispatch_backward(cfg: Config, plan_arena, d_recv, dx, dev_status, stream=None) -> None:
+    _check("moonep_dispatch_backward", _lib.moonep_dispatch_backward(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(d_recv), _ptr(dx), _ptr(dev_status),
+        _stream(stream)))
+
+
+def moonep_prefetch_weight(cfg: Config, plan_arena, weights, rep_weights, W: int, dev_status,
+                           stream=None) -> None:
+    _check("moonep_prefetch_weight", _lib.moonep_prefetch_weight(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(weights), _ptr(rep_weights), int(W),
         _ptr(dev_status), _stream(stream)))
 
 

@@ -110,7 +110,7 @@ combine_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict_
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    const float my_w = lane < K ? (gates ? __ldg(gates + t * K + lane) : 1.f) : 0.f;
     for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
       float acc[U][8];
 #pragma unroll
@@ -166,7 +166,7 @@ combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restric
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    const float my_w = lane < K ? (gates ? __ldg(gates + t * K + lane) : 1.f) : 0.f;
     int rows[KMAX];
     float ws[KMAX];
 #pragma unroll
@@ -222,7 +222,7 @@ combine_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__res
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? gates[t * K + lane] : 0.f;
+    const float my_w = lane < K ? (gates ? gates[t * K + lane] : 1.f) : 0.f;
     for (int64_t h0 = 0; h0 < H; h0 += 32) {
       const int64_t h = h0 + lane;
       float acc = 0.f;
@@ -251,7 +251,7 @@ combine_bwd_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restr
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    const float my_w = lane < K ? (gates ? __ldg(gates + t * K + lane) : 1.f) : 0.f;
     const uint4 *g = dout + t * nvec;
     float my_dg = 0.f;
     for (int k = 0; k < K; k++) {
@@ -312,7 +312,7 @@ combine_bwd_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__res
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? __ldg(gates + t * K + lane) : 0.f;
+    const float my_w = lane < K ? (gates ? __ldg(gates + t * K + lane) : 1.f) : 0.f;
     int rows[KMAX];
     float ws[KMAX], part[KMAX];
 #pragma unroll
@@ -381,7 +381,7 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
   for (int64_t t = warp_g; t < T; t += nwarps) {
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
-    const float my_w = lane < K ? gates[t * K + lane] : 0.f;
+    const float my_w = lane < K ? (gates ? gates[t * K + lane] : 1.f) : 0.f;
     float my_dg = 0.f;
     for (int k = 0; k < K; k++) {
       const int row = __shfl_sync(0xffffffffu, my_slot, k);
@@ -490,6 +490,93 @@ reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__
         o.w = pack_bf16x2(acc[u][6], acc[u][7]);
         hrow[v] = o;
       }
+    }
+  }
+}
+
+// -------------------------------------------------------- prefetch_weight ---
+// Work units: (replicated expert, warp-chunk of 32*U column vectors).  The home
+// weight vectors are read once and stored into every local replica slot of the
+// expert (the expert's pieces with a weight slot).
+template <int U>
+__global__ void __launch_bounds__(kThreads)
+prefetch_weight_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
+                           const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
+                           const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
+                           const uint4 *__restrict__ w, uint4 *__restrict__ rep_w, int64_t nvec,
+                           int R, int E, int B, int PMAX, int32_t *status) {
+  int64_t n_exp = scalars[S_N_REPLICATED];
+  if (n_exp < 0 || n_exp > E) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+    n_exp = 0;
+  }
+  const int64_t per_exp = (nvec + 32 * U - 1) / (32 * U);
+  const int64_t total = n_exp * per_exp;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t wk = warp_g; wk < total; wk += nwarps) {
+    const int e = replicated[wk / per_exp];
+    const int64_t v0 = (wk % per_exp) * 32 * U;
+    const int b = e >= 0 && e < E ? pbeg[e] : 0, en = e >= 0 && e < E ? pend[e] : -1;
+    if (e < 0 || e >= E || b < 0 || en > PMAX || en < b) {
+      if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+      continue;
+    }
+    const uint4 *src = w + (int64_t)e * nvec;
+    uint4 q[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = v0 + u * 32 + lane;
+      q[u] = v < nvec ? __ldcs(src + v) : make_uint4(0, 0, 0, 0);
+    }
+    for (int pc = b; pc < en; pc++) {
+      const int ws = pwslot[pc], rk = prank[pc];
+      if (ws < 0) continue;
+      if (ws >= B || rk < 0 || rk >= R) {
+        if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+        continue;
+      }
+      uint4 *dst = rep_w + ((int64_t)rk * B + ws) * nvec;
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) dst[v] = q[u];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+prefetch_weight_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
+                              const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
+                              const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
+                              const uint16_t *__restrict__ w, uint16_t *__restrict__ rep_w, int64_t W,
+                              int R, int E, int B, int PMAX, int32_t *status) {
+  int64_t n_exp = scalars[S_N_REPLICATED];
+  if (n_exp < 0 || n_exp > E) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+    n_exp = 0;
+  }
+  const int64_t total = n_exp * W;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {
+    const int e = replicated[q / W];
+    const int64_t c = q % W;
+    const int b = e >= 0 && e < E ? pbeg[e] : 0, en = e >= 0 && e < E ? pend[e] : -1;
+    if (e < 0 || e >= E || b < 0 || en > PMAX || en < b) {
+      set_status(status, MOONEP_DEV_BAD_PLAN);
+      continue;
+    }
+    const uint16_t v = w[(int64_t)e * W + c];
+    for (int pc = b; pc < en; pc++) {
+      const int ws = pwslot[pc], rk = prank[pc];
+      if (ws < 0) continue;
+      if (ws >= B || rk < 0 || rk >= R) {
+        set_status(status, MOONEP_DEV_BAD_PLAN);
+        continue;
+      }
+      rep_w[((int64_t)rk * B + ws) * W + c] = v;
     }
   }
 }
@@ -659,6 +746,61 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], rep_grads, home_grads, P_elems, (int)d.R,
         (int)d.E, (int)d.B, (int)d.PMAX, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
+                                                    const void *plan_arena, const uint16_t *d_recv,
+                                                    uint16_t *dx, int32_t *dev_status,
+                                                    moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!d_recv || !dx || !aligned256(plan_arena)) return MOONEP_ERR_INVALID_ARG;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS;
+  // the combine kernels with unit weights: fmaf(1, y, acc) rounds like acc + y
+  if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx) && d.K <= 8) {
+    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
+        reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx)) {
+    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+        P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
+        reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, nrows, dev_status);
+  } else {
+    combine_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], d_recv, nullptr, dx,
+                                                              T, (int)d.K, d.H, nrows, dev_status);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
+                                                  const void *plan_arena, const uint16_t *weights,
+                                                  uint16_t *rep_weights, int64_t W,
+                                                  int32_t *dev_status, moonep_stream_t stream) {
+  Dims d;
+  if (!make_dims(cfg, &d) || !plan_arena || !dev_status || W < 1) return MOONEP_ERR_INVALID_ARG;
+  if (!weights || (d.B > 0 && !rep_weights) || !aligned256(plan_arena))
+    return MOONEP_ERR_INVALID_ARG;
+  if (d.B == 0) return MOONEP_OK;  // no replica slots: every duplicate reads remotely
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const unsigned grid = (unsigned)num_sms() * 8;
+  if (W % 8 == 0 && aligned16(weights) && aligned16(rep_weights)) {
+    prefetch_weight_vec_kernel<4><<<grid, kThreads, 0, st>>>(
+        P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
+        P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(weights),
+        reinterpret_cast<uint4 *>(rep_weights), W / 8, (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX,
+        dev_status);
+  } else {
+    prefetch_weight_scalar_kernel<<<grid, kThreads, 0, st>>>(
+        P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
+        P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], weights, rep_weights, W, (int)d.R, (int)d.E,
+        (int)d.B, (int)d.PMAX, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
