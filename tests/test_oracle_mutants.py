@@ -24,8 +24,8 @@ MUTANTS = {
                                 "for (e = d * L; e < (d + 1) * L && 0; e++) {\n      int64_t idx = d * E + nseg;"),
     "weight_slot_off_by_one": ("out->piece_wslot[n_piece] = (int32_t)j;",
                                "out->piece_wslot[n_piece] = (int32_t)(j + 1 < B ? j + 1 : j);"),
-    "combine_drops_last_k": ("for (int64_t k = 0; k < K; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc",
-                             "for (int64_t k = 0; k < K - 1; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc"),
+    "combine_drops_last_k": ("for (int64_t k = 0; k < K; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc = fmaf",
+                             "for (int64_t k = 0; k < K - 1; k++) {\n        int64_t row = slot_of[t * K + k];\n        acc = fmaf"),
     "backward_without_gate": ("float prod = w * g;", "float prod = g;"),
     "reduce_skips_first_piece": ("acc = acc + orc_bf16_to_f32(rep[slot * P + q]);",
                                  "if (i > 0) acc = acc + orc_bf16_to_f32(rep[slot * P + q]);"),
