@@ -479,6 +479,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
     ap.add_argument("--sweep", action="store_true", help="maxvio sweep of the workload shape")
+    ap.add_argument("--compare-copy", action="store_true",
+                    help="zero-copy dispatch+combine against the copy-through-buffer path")
     ap.add_argument("--scale-s", type=int, default=1, help="divide S (tokens/rank) by this (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -516,6 +518,8 @@ def main():
                                 P=max(8, (w.P or 2048 * w.H) // args.scale_s))
     if args.sweep:
         return run_sweep(args, w, device)
+    if args.compare_copy:
+        return run_compare_copy(args, w, device)
     mv = args.maxvio if args.maxvio is not None else w.maxvio[0]
     layer = Layer(w, mv, args.seed + rank, device)
     total_ms, per, clocks, st = time_steps(layer, args.steps, args.warmup, barrier)
@@ -586,6 +590,55 @@ def main():
     if pg:
         pg.barrier()
         pg.destroy_process_group()
+    return 0
+
+
+def run_compare_copy(args, w, device):
+    """Forward layer with zero copy (moonep_dispatch / moonep_combine) against the
+    zero_copy=False path (rows land in a comm buffer in arrival order, then a permute;
+    permute back before combine).  Same results, same useful bytes."""
+    import torch
+    me = __import__("token_dispatch_moonep_b200")
+    mv = args.maxvio if args.maxvio is not None else w.maxvio[0]
+    layer = Layer(w, mv, args.seed, device, with_backward=False, host_inputs=False)
+    c, T, K, N = layer.cfg, w.R * w.S, w.K, w.R * w.S * w.K
+    comm = torch.empty_like(layer.recv)
+    cidx = torch.empty(N + w.R, dtype=torch.int32, device=device)
+    st = layer.status
+    zc = [("dispatch", lambda: me.moonep_dispatch(c, layer.arena, layer.x, layer.recv, st)),
+          ("combine", lambda: me.moonep_combine(c, layer.arena, layer.recv, layer.gates, layer.out,
+                                                st))]
+    vb = [("dispatch_via_buffer", lambda: me.moonep_dispatch_via_buffer(
+              c, layer.arena, layer.x, comm, cidx, layer.recv, st)),
+          ("combine_via_buffer", lambda: me.moonep_combine_via_buffer(
+              c, layer.arena, layer.recv, layer.gates, cidx, comm, layer.out, st))]
+    me.moonep_plan(c, layer.idx, layer.arena, layer.ws, st)
+    res = {}
+    for name, ops in (("zero_copy", zc), ("via_buffer", vb)):
+        for _ in range(args.warmup):
+            for _, fn in ops:
+                fn()
+        torch.cuda.synchronize()
+        n = max(20, args.steps // 4)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(n)]
+        for i in range(n):
+            ev[i][0].record()
+            for j, (_, fn) in enumerate(ops):
+                fn()
+                ev[i][j + 1].record()
+        torch.cuda.synchronize()
+        per = {op: statistics.median(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n))
+               for j, (op, _) in enumerate(ops)}
+        res[name] = per
+    b = algorithmic_bytes(w.R, w.S, K, w.H)
+    useful = b["dispatch"] + b["combine"]
+    zc_ms, vb_ms = sum(res["zero_copy"].values()), sum(res["via_buffer"].values())
+    print(json.dumps({"compare": "zero_copy vs via_buffer", "workload": w.name,
+                      "maxvio": round(layer.maxvio, 4), "zero_copy_ms": res["zero_copy"],
+                      "via_buffer_ms": res["via_buffer"],
+                      "zero_copy_GBs": useful / (zc_ms * 1e-3) / 1e9,
+                      "via_buffer_GBs": useful / (vb_ms * 1e-3) / 1e9,
+                      "time_ratio": vb_ms / zc_ms, "device_status": int(st.item())}), flush=True)
     return 0
 
 

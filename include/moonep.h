@@ -251,6 +251,32 @@ MOONEP_API moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
                                                   uint16_t *rep_weights, int64_t W,
                                                   int32_t *dev_status, moonep_stream_t stream);
 
+/* The zero_copy=False comparison path ("MoonshotAI/MoonEP 딥다이브" §6: the
+ * zero_copy=True option removes a copy; §8 exercise D measures the epilogue
+ * copy it saves).  Rows first land in a per-rank communication buffer `comm`
+ * (bf16 [R*NvS, H]) in arrival order, then a permute copies them into the
+ * expert-ordered `recv`.  The result is bit-identical to moonep_dispatch; only
+ * the extra copy differs.
+ *   comm_index  device int32 [R*S*K + R]: on return the comm row of every pair
+ *               (order inside a rank unspecified); the last R words are counters
+ *   requires H % 8 == 0 and 16-byte aligned x, comm, recv (else UNSUPPORTED).
+ * Enqueues a 4-byte-per-rank memset and three kernels. */
+MOONEP_API moonep_status_t moonep_dispatch_via_buffer(const moonep_config_t *cfg,
+                                                      const void *plan_arena, const uint16_t *x,
+                                                      uint16_t *comm, int32_t *comm_index,
+                                                      uint16_t *recv, int32_t *dev_status,
+                                                      moonep_stream_t stream);
+
+/* The matching combine of the comparison path: the expert outputs y (expert
+ * order) are permuted back into `comm` at the rows comm_index gives (as left
+ * by moonep_dispatch_via_buffer), then combined from there.  Bit-identical to
+ * moonep_combine. */
+MOONEP_API moonep_status_t moonep_combine_via_buffer(const moonep_config_t *cfg,
+                                                     const void *plan_arena, const uint16_t *y,
+                                                     const float *gates, const int32_t *comm_index,
+                                                     uint16_t *comm, uint16_t *out,
+                                                     int32_t *dev_status, moonep_stream_t stream);
+
 /* Static description of a status code. */
 MOONEP_API const char *moonep_status_string(moonep_status_t status);
 

@@ -304,3 +304,37 @@ def test_prefetch_weight_matches_oracle(shape):
     assert status.item() == 0
     ref = oracle.prefetch_weight(ocfg, ot, w, before)
     assert np.array_equal(to_np(rep), ref)
+
+
+@pytest.mark.parametrize("shape", [(8, 32, 4, 256, 512, 1), (4, 16, 8, 33, 136, 16),
+                                   (8, 64, 8, 1200, 1032, 1), (64, 256, 8, 8, 64, 1)])
+def test_copy_through_buffer_path_equals_zero_copy(shape):
+    """zero_copy=False: land in a comm buffer in arrival order, permute, and back."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S, H, A = shape
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, H, align=A, seed=16)
+    NvS = int(ot["nvs"][0])
+    N = R * S * K
+    x = make_x(R, S, H, seed=16).reshape(R * S, H)
+    ref_recv = oracle.dispatch(ocfg, ot["slot_of"], x, np.full((R * NvS, H), POISON, np.uint16))
+    comm = torch.zeros((R * NvS, H), dtype=torch.int16, device="cuda")
+    cidx = torch.full((N + R,), -5, dtype=torch.int32, device="cuda")
+    recv = torch.full((R * NvS, H), POISON - 65536, dtype=torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    me.moonep_dispatch_via_buffer(cfg, arena, to_dev(x), comm, cidx, recv, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert np.array_equal(to_np(recv), ref_recv)
+    ci = to_np(cidx)[:N]
+    # every rank's S*K comm rows are used exactly once, by pairs sent to that rank
+    assert np.array_equal(np.sort(ci), np.sort(
+        (np.arange(R)[:, None] * NvS + np.arange(S * K)[None, :]).ravel()))
+    assert ((ci // NvS) == (ot["slot_of"] // NvS)).all()
+    y = normal_bf16((R * NvS, H), seed=17, stream=9)
+    w = make_gates(R, S, K, seed=17)
+    out = torch.empty((R * S, H), dtype=torch.int16, device="cuda")
+    me.moonep_combine_via_buffer(cfg, arena, to_dev(y), to_dev(w.ravel()), cidx, comm, out, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert np.array_equal(to_np(out), oracle.combine(ocfg, ot["slot_of"], y, w))

@@ -18,6 +18,8 @@ The functions keep the C names::
     moonep_reduce_grad(cfg, plan_arena, rep_grads, home_grads, P, dev_status, stream=None)
     moonep_dispatch_backward(cfg, plan_arena, d_recv, dx, dev_status, stream=None)
     moonep_prefetch_weight(cfg, plan_arena, weights, rep_weights, W, dev_status, stream=None)
+    moonep_dispatch_via_buffer(cfg, plan_arena, x, comm, comm_index, recv, dev_status, stream=None)
+    moonep_combine_via_buffer(cfg, plan_arena, y, gates, comm_index, comm, out, dev_status, stream=None)
 
 Tensor arguments are device tensors (bf16 tensors may be ``torch.bfloat16``
 or ``int16``/``uint16`` views); raw integer device addresses are accepted too.
@@ -133,6 +135,10 @@ _lib.moonep_dispatch_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_dispatch_backward.restype = _ST
 _lib.moonep_prefetch_weight.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
 _lib.moonep_prefetch_weight.restype = _ST
+_lib.moonep_dispatch_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
+_lib.moonep_dispatch_via_buffer.restype = _ST
+_lib.moonep_combine_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
+_lib.moonep_combine_via_buffer.restype = _ST
 _lib.moonep_status_string.argtypes = [_ST]
 _lib.moonep_status_string.restype = ctypes.c_char_p
 
@@ -269,6 +275,20 @@ def moonep_prefetch_weight(cfg: Config, plan_arena, weights, rep_weights, W: int
     _check("moonep_prefetch_weight", _lib.moonep_prefetch_weight(
         ctypes.byref(cfg), _ptr(plan_arena), _ptr(weights), _ptr(rep_weights), int(W),
         _ptr(dev_status), _stream(stream)))
+
+
+def moonep_dispatch_via_buffer(cfg: Config, plan_arena, x, comm, comm_index, recv, dev_status,
+                               stream=None) -> None:
+    _check("moonep_dispatch_via_buffer", _lib.moonep_dispatch_via_buffer(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(x), _ptr(comm), _ptr(comm_index), _ptr(recv),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moonep_combine_via_buffer(cfg: Config, plan_arena, y, gates, comm_index, comm, out, dev_status,
+                              stream=None) -> None:
+    _check("moonep_combine_via_buffer", _lib.moonep_combine_via_buffer(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(y), _ptr(gates), _ptr(comm_index), _ptr(comm),
+        _ptr(out), _ptr(dev_status), _stream(stream)))
 
 
 # ---------------------------------------------------------- allocation help ---

@@ -494,6 +494,89 @@ reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__
   }
 }
 
+// ------------------------------------------------ copy-through-buffer mode ---
+// The zero_copy=False comparison path: pairs first land in a per-rank
+// communication buffer in arrival order, then a permute copies them into the
+// expert-ordered dispatch buffer (and back out before combine).
+//
+// comm_place: 64 tokens per CTA; each pair reserves its row in its destination
+// rank's part of the buffer: a shared-memory count per destination, one global
+// reservation per (CTA, destination), then the CTA-local position.  Arrival
+// order inside a rank is unspecified (as it is for a real receiver).
+constexpr int kCommTokensPerBlock = 64;
+
+__global__ void __launch_bounds__(512)
+comm_place_kernel(const int32_t *__restrict__ slot_of, int32_t *__restrict__ comm_index,
+                  int32_t *__restrict__ counters, int64_t T, int K, int R, int64_t NvS,
+                  int32_t *status) {
+  extern __shared__ int cs[];  // [R] local counts, then [R] global bases
+  int *cnt = cs, *base = cs + R;
+  for (int d = threadIdx.x; d < R; d += blockDim.x) cnt[d] = 0;
+  __syncthreads();
+  const int64_t t0 = (int64_t)blockIdx.x * kCommTokensPerBlock;
+  const int64_t np = (int64_t)kCommTokensPerBlock * K;
+  const int64_t nrows = (int64_t)R * NvS;
+  for (int64_t i = threadIdx.x; i < np; i += blockDim.x) {
+    const int64_t p = t0 * K + i;
+    if (p >= T * K) break;
+    const int row = slot_of[p];
+    if (row < 0 || row >= nrows) continue;
+    atomicAdd(&cnt[row / NvS], 1);
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < R; d += blockDim.x) {
+    base[d] = cnt[d] ? atomicAdd(&counters[d], cnt[d]) : 0;
+    cnt[d] = 0;
+  }
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < np; i += blockDim.x) {
+    const int64_t p = t0 * K + i;
+    if (p >= T * K) break;
+    const int row = slot_of[p];
+    if (row < 0 || row >= nrows) {
+      comm_index[p] = -1;
+      continue;
+    }
+    const int d = (int)(row / NvS);
+    const int pos = base[d] + atomicAdd(&cnt[d], 1);
+    if (pos >= NvS) {  // impossible when every rank receives S*K pairs
+      set_status(status, MOONEP_DEV_BAD_PLAN);
+      comm_index[p] = -1;
+      continue;
+    }
+    comm_index[p] = (int32_t)(d * NvS + pos);
+  }
+}
+
+// dst[dst_index[p]] = src[src_index[p]] for every pair, one warp per pair (rows of nvec vectors)
+__global__ void __launch_bounds__(kThreads)
+permute_rows_kernel(const int32_t *__restrict__ src_index, const int32_t *__restrict__ dst_index,
+                    const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t npairs,
+                    int64_t nvec, int64_t nrows) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (int64_t p = warp_g; p < npairs; p += nwarps) {
+    const int a = __ldg(src_index + p), b = __ldg(dst_index + p);
+    if (a < 0 || b < 0 || a >= nrows || b >= nrows) continue;
+    const uint4 *s = src + (int64_t)a * nvec;
+    uint4 *d = dst + (int64_t)b * nvec;
+    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * 4) {
+      uint4 q[4];
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) q[u] = __ldcs(s + v);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const int64_t v = v0 + u * 32 + lane;
+        if (v < nvec) d[v] = q[u];
+      }
+    }
+  }
+}
+
 // -------------------------------------------------------- prefetch_weight ---
 // Work units: (replicated expert, warp-chunk of 32*U column vectors).  The home
 // weight vectors are read once and stored into every local replica slot of the
@@ -802,6 +885,79 @@ extern "C" moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], weights, rep_weights, W, (int)d.R, (int)d.E,
         (int)d.B, (int)d.PMAX, dev_status);
   }
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+namespace {
+unsigned pair_grid(int64_t npairs) {
+  int64_t blocks = (npairs + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int64_t cap = (int64_t)num_sms() * 64;
+  if (blocks > cap) blocks = cap;
+  return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+}  // namespace
+
+extern "C" moonep_status_t moonep_dispatch_via_buffer(const moonep_config_t *cfg,
+                                                      const void *plan_arena, const uint16_t *x,
+                                                      uint16_t *comm, int32_t *comm_index,
+                                                      uint16_t *recv, int32_t *dev_status,
+                                                      moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!x || !comm || !comm_index || !recv || !aligned256(plan_arena)) return MOONEP_ERR_INVALID_ARG;
+  if (d.H % 8 != 0 || !aligned16(x) || !aligned16(comm) || !aligned16(recv))
+    return MOONEP_ERR_UNSUPPORTED;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS, N = T * d.K;
+  int32_t *counters = comm_index + N;
+  if (cudaMemsetAsync(counters, 0, sizeof(int32_t) * d.R, st) != cudaSuccess) return MOONEP_ERR_CUDA;
+  const unsigned blocks = (unsigned)((T + kCommTokensPerBlock - 1) / kCommTokensPerBlock);
+  comm_place_kernel<<<blocks, 512, 2 * d.R * sizeof(int), st>>>(P.f[F_SLOT_OF], comm_index, counters,
+                                                                 T, (int)d.K, (int)d.R, d.NvS,
+                                                                 dev_status);
+  // the sender writes rows into the receivers' communication buffers
+  dispatch_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+      comm_index, reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(comm), T, (int)d.K,
+      d.H / 8, nrows, dev_status);
+  // the receiver permutes them into expert order
+  permute_rows_kernel<<<pair_grid(N), kThreads, 0, st>>>(
+      comm_index, P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(comm),
+      reinterpret_cast<uint4 *>(recv), N, d.H / 8, nrows);
+  return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+
+extern "C" moonep_status_t moonep_combine_via_buffer(const moonep_config_t *cfg,
+                                                     const void *plan_arena, const uint16_t *y,
+                                                     const float *gates, const int32_t *comm_index,
+                                                     uint16_t *comm, uint16_t *out,
+                                                     int32_t *dev_status, moonep_stream_t stream) {
+  Dims d;
+  if (!data_dims(cfg, &d) || !plan_arena || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  const int64_t T = d.R * d.S;
+  if (T == 0) return MOONEP_OK;
+  if (!y || !gates || !comm_index || !comm || !out || !aligned256(plan_arena))
+    return MOONEP_ERR_INVALID_ARG;
+  if (d.H % 8 != 0 || !aligned16(y) || !aligned16(comm) || !aligned16(out))
+    return MOONEP_ERR_UNSUPPORTED;
+  PlanPtrs P = plan_ptrs(d, plan_arena);
+  cudaStream_t st = to_cuda(stream);
+  const int64_t nrows = d.R * d.NvS, N = T * d.K;
+  // the expert ranks permute their outputs back into arrival order
+  permute_rows_kernel<<<pair_grid(N), kThreads, 0, st>>>(
+      P.f[F_SLOT_OF], comm_index, reinterpret_cast<const uint4 *>(y), reinterpret_cast<uint4 *>(comm),
+      N, d.H / 8, nrows);
+  // and the source ranks combine from the communication buffer
+  if (d.K <= 8)
+    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+        comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
+        (int)d.K, d.H / 8, nrows, dev_status);
+  else
+    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+        comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
+        (int)d.K, d.H / 8, nrows, dev_status);
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
