@@ -78,21 +78,31 @@ __device__ __forceinline__ void st_release(int32_t *p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ int ld_relaxed(const int32_t *p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Warp-wide bounded wait until flags[0, n) all equal v.  False on timeout.
+// Polls with relaxed loads (independent, so they overlap) and fences once after.
 __device__ bool warp_wait_all(const int32_t *flags, int64_t n, int v, long long limit_ns) {
   const int lane = threadIdx.x & 31;
   const unsigned long long t0 = now_ns();
   int64_t from = 0;  // flags before `from` are known to have arrived
   for (;;) {
     bool mine = true;
-    for (int64_t c = from + lane; c < n && c < from + 1024; c += 32) mine &= ld_acquire(flags + c) == v;
+    for (int64_t c = from + lane; c < n && c < from + 1024; c += 32) mine &= ld_relaxed(flags + c) == v;
     if (__all_sync(0xffffffffu, mine)) {
       from += 1024;
-      if (from >= n) return true;
+      if (from >= n) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        return true;
+      }
       continue;
     }
     if ((long long)(now_ns() - t0) > limit_ns) return false;
-    __nanosleep(64);
+    __nanosleep(32);
   }
 }
 
@@ -458,17 +468,8 @@ __device__ int solve_core(const PlanArgs &a, const SolveSmem &m) {
   for (int h = tid; h < R; h += nt)
     if (m.ntot[h] > NvS) m.misc[1] = 1;
   __syncthreads();
-  return m.misc[1] ? kStCapacity : 0;
-}
-
-// Every other plan table (after the done flag; placement does not read them).
-__device__ void solve_outputs(const PlanArgs &a, const SolveSmem &m) {
-  const Dims &d = a.d;
-  const PlanPtrs &P = a.P;
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
-  const int n_recv = m.misc[0], n_piece = m.misc[3];
-
+  // segments per rank (published with the placement tables: the workers fill
+  // the unused segment entries and replica slots from it)
   for (int i = tid; i < n_recv; i += nt) {  // first and last piece of each receiver
     const int ef = upper_bound_i(m.oend, E, m.rbase[i]);
     m.rfirst[i] = ef < E ? m.npc[ef] + (i - m.i0[ef]) : 0;
@@ -478,6 +479,19 @@ __device__ void solve_outputs(const PlanArgs &a, const SolveSmem &m) {
   }
   for (int h = tid; h < R; h += nt)
     if (m.ridx[h] < 0) m.nseg[h] = L;
+  __syncthreads();
+  for (int h = tid; h < R; h += nt) P.f[F_N_SEG][h] = m.nseg[h];
+  return m.misc[1] ? kStCapacity : 0;
+}
+
+// Every other plan table (after the done flag; placement does not read them).
+__device__ void solve_outputs(const PlanArgs &a, const SolveSmem &m) {
+  const Dims &d = a.d;
+  const PlanPtrs &P = a.P;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
+  const int n_piece = m.misc[3];
+
   for (int e = tid; e < E; e += nt) m.flag[e] = 0;
   __syncthreads();
   for (int pid = tid; pid < n_piece; pid += nt) {
@@ -518,21 +532,6 @@ __device__ void solve_outputs(const PlanArgs &a, const SolveSmem &m) {
     P.f[F_RANK_LOAD][h] = ld;
     P.f[F_OVERFLOW][h] = ld > SK ? ld - SK : 0;
     P.f[F_DEFICIT][h] = ld < SK ? SK - ld : 0;
-    P.f[F_N_SEG][h] = m.nseg[h];
-  }
-  for (int64_t q = tid; q < d.R * d.E; q += nt) {  // unused segment entries
-    const int h = (int)(q / E), i = (int)(q % E);
-    if (i >= m.nseg[h]) {
-      P.f[F_SEG_EXPERT][q] = -1;
-      P.f[F_SEG_START][q] = 0;
-      P.f[F_SEG_LEN][q] = 0;
-      P.f[F_SEG_KIND][q] = -1;
-      P.f[F_SEG_WSLOT][q] = -1;
-    }
-  }
-  for (int64_t q = tid; q < d.R * d.B; q += nt) {  // free replica slots
-    const int h = (int)(q / B), j = (int)(q % B);
-    if (j >= m.nseg[h] - L) P.f[F_REP_EXPERT][q] = -1;
   }
   __syncthreads();
   for (int e = tid; e < E; e += nt) m.i0[e] = m.flag[e];  // keep the flags across the scan
@@ -733,6 +732,24 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
     int32_t *slot_of = a.P.f[F_SLOT_OF];
     for (int64_t k = wk; k < a.nc; k += W)
       for (int64_t p = k * a.ch + tid; p < (k + 1) * a.ch && p < d.N; p += kPlanThreads) slot_of[p] = -1;
+  }
+
+  // unused segment entries and free replica slots (from the published n_seg)
+  if (!invalid) {
+    const int L = (int)d.L, B = (int)d.B;
+    for (int h = wk; h < (int)d.R; h += W) {
+      const int ns = __ldcg(a.P.f[F_N_SEG] + h);
+      for (int i = ns + tid; i < E; i += kPlanThreads) {
+        const int64_t q = (int64_t)h * E + i;
+        a.P.f[F_SEG_EXPERT][q] = -1;
+        a.P.f[F_SEG_START][q] = 0;
+        a.P.f[F_SEG_LEN][q] = 0;
+        a.P.f[F_SEG_KIND][q] = -1;
+        a.P.f[F_SEG_WSLOT][q] = -1;
+      }
+      for (int j = (ns - L) + tid; j < B; j += kPlanThreads)
+        if (j >= 0) a.P.f[F_REP_EXPERT][(int64_t)h * B + j] = -1;
+    }
   }
 
   // rows that hold no pair: everything after an invalid plan, padding when A > 1
