@@ -38,7 +38,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moonep.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"libmoonep.so is not built ({LIB_PATH}); run `python -m token_dispatch_moonep_b200.build` "
+        f"libmoonep.so is not built ({LIB_PATH}); run `python token_dispatch_moonep_b200/build.py` "
         "(nvcc, sm_100a). There is no fallback implementation.")
 
 _lib = ctypes.CDLL(LIB_PATH)
