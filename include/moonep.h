@@ -103,7 +103,8 @@ typedef struct moonep_plan_view {
   int32_t *seg_len;            /* [R*E] rows */
   int32_t *seg_kind;           /* [R*E] MOONEP_SEG_* (-1 unused) */
   int32_t *seg_wslot;          /* [R*E] replica weight slot, -1 for native / remote */
-  int32_t *piece_expert;       /* [P_MAX] replica pieces in overflow-stream order */
+  int32_t *piece_expert;       /* [P_MAX] replica pieces in overflow-stream order; entries of
+                                  every piece table at index >= scalars[0] are unspecified */
   int32_t *piece_rank;         /* [P_MAX] receiving rank */
   int32_t *piece_start;        /* [P_MAX] first row within the receiving rank */
   int32_t *piece_len;          /* [P_MAX] rows */
@@ -112,7 +113,8 @@ typedef struct moonep_plan_view {
   int32_t *expert_piece_begin; /* [E] pieces of expert e are [begin, end) */
   int32_t *expert_piece_end;   /* [E] */
   int32_t *rep_expert;         /* [R*budget] expert in weight slot j of rank d, -1 if free */
-  int32_t *replicated_experts; /* [E] experts with >= 1 local replica, ascending; count in scalars[3] */
+  int32_t *replicated_experts; /* [E] experts with >= 1 local replica, ascending; count in
+                                  scalars[3], later entries unspecified */
   int32_t *scalars;            /* [8] 0 n_piece, 1 n_remote, 2 n_local_pieces, 3 n_replicated */
   int64_t nvs;                 /* rows per rank */
   int32_t max_pieces;          /* P_MAX */

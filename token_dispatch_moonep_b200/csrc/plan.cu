@@ -332,49 +332,39 @@ __device__ int solve_core(const PlanArgs &a, const SolveSmem &m) {
     }
   }
   __syncthreads();
-  // overflow / deficit bases, receiver compaction
-  if (R <= 32) {
-    if (warp == 0) {
-      const int ld = lane < R ? m.load[lane] : SK;
-      const int ov = ld > SK ? ld - SK : 0;
-      const int df = ld < SK ? SK - ld : 0;
-      const int rf = df > 0 ? 1 : 0;
-      const int iov = warp_incl_scan(ov), idf = warp_incl_scan(df), irf = warp_incl_scan(rf);
-      if (lane < R) {
-        m.over[lane] = iov - ov;
-        m.def[lane] = idf - df;
-        m.ridx[lane] = rf ? irf - 1 : -1;
-        if (rf) {
-          m.rrank[irf - 1] = lane;
-          m.rbase[irf - 1] = idf - df;
-          m.rend[irf - 1] = idf;
-        }
-      }
-      if (lane == 31) m.misc[0] = irf;
-    }
-  } else {
-    for (int h = tid; h < R; h += nt) {
+  // overflow / deficit bases, receiver compaction: one warp, ceil(R/32)
+  // consecutive ranks per lane, three warp scans
+  if (warp == 0) {
+    const int per = (R + 31) / 32;
+    const int h0 = lane * per < R ? lane * per : R;
+    const int h1 = h0 + per < R ? h0 + per : R;
+    int sov = 0, sdf = 0, srf = 0;
+    for (int h = h0; h < h1; h++) {
       const int ld = m.load[h];
-      m.over[h] = ld > SK ? ld - SK : 0;
-      m.def[h] = ld < SK ? SK - ld : 0;
-      m.tmp[h] = m.def[h];
-      m.ridx[h] = m.def[h] > 0 ? 1 : 0;
+      sov += ld > SK ? ld - SK : 0;
+      sdf += ld < SK ? SK - ld : 0;
+      srf += ld < SK ? 1 : 0;
     }
-    int *arr[3] = {m.over, m.def, m.ridx};
-    int tot[3];
-    __syncthreads();
-    block_excl_scan<3>(arr, R, m.scratch, tot);
-    for (int h = tid; h < R; h += nt) {
-      if (m.tmp[h] > 0) {
-        const int i = m.ridx[h];
-        m.rrank[i] = h;
-        m.rbase[i] = m.def[h];
-        m.rend[i] = m.def[h] + m.tmp[h];
+    const int iov = warp_incl_scan(sov), idf = warp_incl_scan(sdf), irf = warp_incl_scan(srf);
+    int ov = iov - sov, df = idf - sdf, rf = irf - srf;  // exclusive bases of this lane's ranks
+    for (int h = h0; h < h1; h++) {
+      const int ld = m.load[h];
+      const int o = ld > SK ? ld - SK : 0, dd = ld < SK ? SK - ld : 0;
+      m.over[h] = ov;
+      m.def[h] = df;
+      if (dd > 0) {
+        m.ridx[h] = rf;
+        m.rrank[rf] = h;
+        m.rbase[rf] = df;
+        m.rend[rf] = df + dd;
+        rf++;
       } else {
         m.ridx[h] = -1;
       }
+      ov += o;
+      df += dd;
     }
-    if (tid == 0) m.misc[0] = tot[2];
+    if (lane == 31) m.misc[0] = irf;
   }
   __syncthreads();
   const int n_recv = m.misc[0];
@@ -428,42 +418,50 @@ __device__ int solve_core(const PlanArgs &a, const SolveSmem &m) {
   if (tid == 0) m.misc[3] = n_piece;
   __syncthreads();
 
-  // placement tables
+  // placement tables: per expert, then per piece, one thread each.  The expert
+  // of piece pid is the last e with first-piece id npc[e] <= pid (npc is the
+  // exclusive scan of the piece counts, so that expert has a piece).
   for (int e = tid; e < E; e += nt) {
     const int h = e / L;
-    const int pb = m.npc[e], npc = m.npcn[e];
-    const int ost = m.oend[e] - m.ovf[e];
     a.exp_kept[e] = m.kept[e];
     a.exp_row0[e] = h * NvS + m.nst[e];
-    a.exp_ostart[e] = ost;
-    P.f[F_EXP_PIECE_BEGIN][e] = pb;
-    P.f[F_EXP_PIECE_END][e] = pb + npc;
-    for (int q = 0; q < npc; q++) {
-      const int i = m.i0[e] + q, pid = pb + q;
-      if (pid >= PM || i >= n_recv) break;
-      const int os = ost > m.rbase[i] ? ost : m.rbase[i];
-      const int oe = m.oend[e] < m.rend[i] ? m.oend[e] : m.rend[i];
-      const int dr = m.rrank[i];
-      int start;
-      if (A == 1) {
-        start = m.ntot[dr] + (os - m.rbase[i]);
-      } else {  // earlier pieces of receiver i: from the expert holding rbase up to e-1
-        const int ef = upper_bound_i(m.oend, E, m.rbase[i]);
-        start = m.ntot[dr];
-        if (ef < e) {
-          start += roundup_i(m.oend[ef] - m.rbase[i], A);
-          for (int e2 = ef + 1; e2 < e; e2++) start += roundup_i(m.ovf[e2], A);
-        }
-      }
-      m.pexp[pid] = e;
-      m.precv[pid] = i;
-      m.post[pid] = os;
-      m.plen[pid] = oe - os;
-      m.pst[pid] = start;
-      P.f[F_PIECE_OSTART][pid] = os;
-      a.piece_grow[pid] = dr * NvS + start;
-      if (start + (oe - os) > NvS) m.misc[1] = 1;
+    a.exp_ostart[e] = m.oend[e] - m.ovf[e];
+    P.f[F_EXP_PIECE_BEGIN][e] = m.npc[e];
+    P.f[F_EXP_PIECE_END][e] = m.npc[e] + m.npcn[e];
+  }
+  for (int pid = tid; pid < n_piece; pid += nt) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (m.npc[mid] <= pid) lo = mid; else hi = mid - 1;
     }
+    const int e = lo;
+    const int q = pid - m.npc[e];
+    const int i = m.i0[e] + q;
+    if (q < 0 || q >= m.npcn[e] || i >= n_recv) continue;
+    const int ost = m.oend[e] - m.ovf[e];
+    const int os = ost > m.rbase[i] ? ost : m.rbase[i];
+    const int oe = m.oend[e] < m.rend[i] ? m.oend[e] : m.rend[i];
+    const int dr = m.rrank[i];
+    int start;
+    if (A == 1) {
+      start = m.ntot[dr] + (os - m.rbase[i]);
+    } else {  // earlier pieces of receiver i: from the expert holding rbase up to e-1
+      const int ef = upper_bound_i(m.oend, E, m.rbase[i]);
+      start = m.ntot[dr];
+      if (ef < e) {
+        start += roundup_i(m.oend[ef] - m.rbase[i], A);
+        for (int e2 = ef + 1; e2 < e; e2++) start += roundup_i(m.ovf[e2], A);
+      }
+    }
+    m.pexp[pid] = e;
+    m.precv[pid] = i;
+    m.post[pid] = os;
+    m.plen[pid] = oe - os;
+    m.pst[pid] = start;
+    P.f[F_PIECE_OSTART][pid] = os;
+    a.piece_grow[pid] = dr * NvS + start;
+    if (start + (oe - os) > NvS) m.misc[1] = 1;
   }
   for (int h = tid; h < R; h += nt)
     if (m.ntot[h] > NvS) m.misc[1] = 1;
