@@ -47,37 +47,57 @@ __device__ __forceinline__ int load_slot(const int32_t *slot_of, int64_t t, int 
 }
 
 // ------------------------------------------------------------- dispatch ---
+// One warp per (token, column chunk).  A row of nvec vectors is cut into nch
+// equal chunks of cl <= 32*U vectors; the warp loads its chunk once (U vectors
+// per lane in flight) and stores it to the token's K slots.  Small units keep
+// every SM busy to the end of the launch and a chunk is never a partial loop.
 template <int U>
 __global__ void __launch_bounds__(kThreads)
-dispatch_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ x,
-                    uint4 *__restrict__ recv, int64_t T, int K, int64_t nvec, int64_t nrows,
-                    int32_t *status) {
+dispatch_chunk_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ x,
+                      uint4 *__restrict__ recv, int64_t T, int K, int64_t nvec, int64_t nch,
+                      int64_t cl, int64_t nrows, int32_t *status) {
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
-  for (int64_t t = warp_g; t < T; t += nwarps) {
+  const int64_t nunits = T * nch;
+  for (int64_t w = warp_g; w < nunits; w += nwarps) {
+    const int64_t t = w / nch;
+    const int64_t c0 = (w - t * nch) * cl;
+    const int64_t c1 = c0 + cl < nvec ? c0 + cl : nvec;
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
     const uint4 *src = x + t * nvec;
-    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
-      uint4 buf[U];
+    uint4 buf[U];
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int64_t v = c0 + u * 32 + lane;
+      if (v < c1) buf[u] = __ldcs(src + v);
+    }
+    for (int k = 0; k < K; k++) {
+      const int row = __shfl_sync(0xffffffffu, my_slot, k);
+      if (row < 0) continue;
+      uint4 *dst = recv + (int64_t)row * nvec;
 #pragma unroll
       for (int u = 0; u < U; u++) {
-        const int64_t v = v0 + u * 32 + lane;
-        if (v < nvec) buf[u] = __ldcs(src + v);
-      }
-      for (int k = 0; k < K; k++) {
-        const int row = __shfl_sync(0xffffffffu, my_slot, k);
-        if (row < 0) continue;
-        uint4 *dst = recv + (int64_t)row * nvec;
-#pragma unroll
-        for (int u = 0; u < U; u++) {
-          const int64_t v = v0 + u * 32 + lane;
-          if (v < nvec) dst[v] = buf[u];
-        }
+        const int64_t v = c0 + u * 32 + lane;
+        if (v < c1) dst[v] = buf[u];
       }
     }
   }
 }
+
+// chunking of a row of nvec vectors for dispatch_chunk_kernel<U>
+struct RowChunks {
+  int64_t nch, cl;
+};
+template <int U>
+RowChunks row_chunks(int64_t nvec) {
+  RowChunks r;
+  r.nch = (nvec + 32 * U - 1) / (32 * U);
+  if (r.nch < 1) r.nch = 1;
+  r.cl = (nvec + r.nch - 1) / r.nch;
+  return r;
+}
+constexpr int kDispatchU = 14;
 
 __global__ void __launch_bounds__(kThreads)
 dispatch_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ x,
@@ -753,9 +773,10 @@ extern "C" moonep_status_t moonep_dispatch(const moonep_config_t *cfg, const voi
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS;
   if (d.H % 8 == 0 && aligned16(x) && aligned16(recv)) {
-    dispatch_vec_kernel<8><<<token_grid(T), kThreads, 0, st>>>(
+    const RowChunks rc = row_chunks<kDispatchU>(d.H / 8);
+    dispatch_chunk_kernel<kDispatchU><<<token_grid(T * rc.nch), kThreads, 0, st>>>(
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(recv), T,
-        (int)d.K, d.H / 8, nrows, dev_status);
+        (int)d.K, d.H / 8, rc.nch, rc.cl, nrows, dev_status);
   } else {
     dispatch_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], x, recv, T, (int)d.K,
                                                                d.H, nrows, dev_status);
@@ -887,15 +908,16 @@ extern "C" moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
   if (d.B == 0) return MOONEP_OK;  // no replica slots: every duplicate reads remotely
   PlanPtrs P = plan_ptrs(d, plan_arena);
   cudaStream_t st = to_cuda(stream);
-  const unsigned grid = (unsigned)num_sms() * 8;
   if (W % 8 == 0 && aligned16(weights) && aligned16(rep_weights)) {
-    prefetch_weight_vec_kernel<4><<<grid, kThreads, 0, st>>>(
+    // many small blocks: the block scheduler balances the expert-major units
+    const unsigned grid = (unsigned)num_sms() * 64;
+    prefetch_weight_vec_kernel<8><<<grid, kThreads, 0, st>>>(
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(weights),
         reinterpret_cast<uint4 *>(rep_weights), W / 8, (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX,
         dev_status);
   } else {
-    prefetch_weight_scalar_kernel<<<grid, kThreads, 0, st>>>(
+    prefetch_weight_scalar_kernel<<<(unsigned)num_sms() * 8, kThreads, 0, st>>>(
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], weights, rep_weights, W, (int)d.R, (int)d.E,
         (int)d.B, (int)d.PMAX, dev_status);
@@ -934,9 +956,10 @@ extern "C" moonep_status_t moonep_dispatch_via_buffer(const moonep_config_t *cfg
                                                                  T, (int)d.K, (int)d.R, d.NvS,
                                                                  dev_status);
   // the sender writes rows into the receivers' communication buffers
-  dispatch_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+  const RowChunks rc = row_chunks<kDispatchU>(d.H / 8);
+  dispatch_chunk_kernel<kDispatchU><<<token_grid(T * rc.nch), kThreads, 0, st>>>(
       comm_index, reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(comm), T, (int)d.K,
-      d.H / 8, nrows, dev_status);
+      d.H / 8, rc.nch, rc.cl, nrows, dev_status);
   // the receiver permutes them into expert order
   permute_rows_kernel<<<pair_grid(N), kThreads, 0, st>>>(
       comm_index, P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(comm),

@@ -783,6 +783,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   }
 }
 
+// Largest dynamic shared memory a launch of f may request on device dev (the
+// opt-in limit less the kernel's static shared memory); 0 on error.
+template <typename F>
+int max_dynamic_smem(F f, int dev) {
+  int optin = 0;
+  cudaFuncAttributes fa;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, f) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return optin - (int)fa.sharedSizeBytes;
+}
+
 size_t plan_smem_bytes(const Dims &d) {
   const size_t worker = std::max<size_t>(size_t(kPlanWarps) * d.E,
                                          6 * d.E + 2 * d.PMAX + 4 + 4 * kPlanThreads);
@@ -855,16 +869,21 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   if (!plan_arena || !workspace || !dev_status || (d.N > 0 && !topk_idx))
     return MOONEP_ERR_INVALID_ARG;
   if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOONEP_ERR_CUDA;
   const size_t smem = plan_smem_bytes(d);
-  if (smem > 227 * 1024) return MOONEP_ERR_UNSUPPORTED;
+  const int limit = max_dynamic_smem(plan_kernel, dev);
+  if (limit <= 0) return MOONEP_ERR_CUDA;
+  if (smem > size_t(limit)) return MOONEP_ERR_UNSUPPORTED;
+  // the device's whole limit, so concurrent callers with other configs never
+  // lower it under each other
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) !=
           cudaSuccess)
     return MOONEP_ERR_CUDA;
   // co-resident CTAs: a cooperative launch guarantees they run at the same time
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kPlanThreads, smem) !=
           cudaSuccess)
     return MOONEP_ERR_CUDA;
