@@ -338,3 +338,75 @@ def test_copy_through_buffer_path_equals_zero_copy(shape):
     torch.cuda.synchronize()
     assert status.item() == 0
     assert np.array_equal(to_np(out), oracle.combine(ocfg, ot["slot_of"], y, w))
+
+
+def test_chained_calls_without_host_syncs():
+    """The whole training chain enqueued back to back, one sync at the end.
+
+    Every data kernel is launched with programmatic dependent launch: it may be
+    scheduled while the previous kernel drains and waits on the device for it.
+    Here each call consumes what the call just before it wrote (plan ->
+    prefetch -> dispatch -> combine -> combine-backward -> dispatch-backward ->
+    reduce_grad, and a second plan on new routing), so any read that moved
+    ahead of that wait shows up as a mismatch with the oracle."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S, H, P = 8, 64, 6, 96, 264, 1000
+    cfg, ocfg = configs(R, E, K, S, H=H)
+    dev = torch.device("cuda")
+    NvS = me.moonep_nvs(cfg)
+    idx1, _, _ = make_routing(R, E, K, S, 10.0, seed=21)
+    idx2, _, _ = make_routing(R, E, K, S, 0.5, seed=22)
+    x = make_x(R, S, H, seed=21).reshape(R * S, H)
+    g = make_gates(R, S, K, seed=21)
+    dout = normal_bf16((R * S, H), seed=21, stream=3)
+    w = normal_bf16((E, P), seed=21, stream=4)
+    home0 = normal_bf16((E, P), seed=21, stream=5)
+    arena, ws, st = me.alloc_plan(cfg)
+    arena2, ws2, _ = me.alloc_plan(cfg)
+    idx1_d, idx2_d = to_dev(idx1.ravel().astype(np.int32)), to_dev(idx2.ravel().astype(np.int32))
+    x_d, g_d, dout_d, w_d = to_dev(x), to_dev(g.ravel()), to_dev(dout), to_dev(w)
+    home = to_dev(home0)
+    rep_w = torch.zeros((R * cfg.budget, P), dtype=torch.int16, device=dev)
+    recv = torch.zeros((R * NvS, H), dtype=torch.int16, device=dev)
+    out = torch.zeros((R * S, H), dtype=torch.int16, device=dev)
+    dy = torch.zeros_like(recv)
+    dg = torch.zeros(R * S * K, dtype=torch.float32, device=dev)
+    dx = torch.zeros_like(out)
+    torch.cuda.synchronize()
+    me.moonep_plan(cfg, idx1_d, arena, ws, st)
+    me.moonep_prefetch_weight(cfg, arena, w_d, rep_w, P, st)
+    me.moonep_dispatch(cfg, arena, x_d, recv, st)
+    me.moonep_combine(cfg, arena, recv, g_d, out, st)
+    me.moonep_combine_backward(cfg, arena, dout_d, recv, g_d, dy, dg, st)
+    me.moonep_dispatch_backward(cfg, arena, dy, dx, st)
+    me.moonep_reduce_grad(cfg, arena, rep_w, home, P, st)  # replica "grads" = the prefetched weights
+    me.moonep_plan(cfg, idx2_d, arena2, ws2, st)
+    me.moonep_dispatch(cfg, arena2, out, recv, st)          # second layer reads the first's output
+    torch.cuda.synchronize()
+    assert int(st.item()) & ~me.DEV_BUDGET == 0
+
+    _, ot = oracle.plan(ocfg, idx1)
+    _, ot2 = oracle.plan(ocfg, idx2)
+    ref_rep = oracle.prefetch_weight(ocfg, ot, w, np.zeros((R, cfg.budget, P), np.uint16))
+    ref_recv1 = oracle.dispatch(ocfg, ot["slot_of"], x)
+    ref_out = oracle.combine(ocfg, ot["slot_of"], ref_recv1, g)
+    ref_dy_pairs, ref_dg = oracle.combine_backward(ocfg, ot["slot_of"], dout, ref_recv1, g)
+    ref_dy = np.zeros((R * NvS, H), np.uint16)  # the oracle gives dY per pair: put it in slot order
+    ref_dy[ot["slot_of"]] = ref_dy_pairs.reshape(R * S * K, H)
+    ref_dx = oracle.dispatch_backward(ocfg, ot["slot_of"], ref_dy)
+    ref_home = oracle.reduce_grad(ocfg, ot, ref_rep, home0)
+    ref_recv2 = oracle.dispatch(ocfg, ot2["slot_of"], ref_out)
+
+    def close(got, ref):  # fp32-accumulated results: the tolerance of the other data tests
+        assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+        assert (got == ref).mean() >= 0.999
+
+    assert np.array_equal(to_np(rep_w).reshape(R, cfg.budget, P), ref_rep)  # copies: bit-exact
+    close(to_np(out), ref_out)
+    close(to_np(dy)[ot["slot_of"]], ref_dy[ot["slot_of"]])
+    assert rel_err(to_np(dg).reshape(R * S, K), ref_dg.reshape(R * S, K)) <= TOL
+    close(to_np(dx), ref_dx)
+    close(to_np(home), ref_home)
+    valid = ot2["slot_src"] >= 0
+    close(to_np(recv)[valid], ref_recv2[valid])

@@ -8,6 +8,8 @@
 // (one bf16 per lane) path.
 #include <cuda_bf16.h>
 
+#include <utility>
+
 #include "moonep_internal.cuh"
 
 namespace moonep {
@@ -16,6 +18,29 @@ namespace {
 
 constexpr int kWarpsPerBlock = 8;
 constexpr int kThreads = kWarpsPerBlock * 32;
+
+// Programmatic dependent launch.  Every kernel here is launched with
+// programmatic stream serialisation, so the GPU may start it while the kernel
+// before it in the stream drains; its first instruction waits until that
+// kernel has completed and its memory is visible, so no read or write moves
+// ahead of it.  This hides most of the launch gap between back-to-back kernels.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+            Args &&...args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(block);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);  // errors: cudaGetLastError
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -56,6 +81,7 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_chunk_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ x,
                       uint4 *__restrict__ recv, int64_t T, int K, int64_t nvec, int64_t nch,
                       int64_t cl, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -103,6 +129,7 @@ __global__ void __launch_bounds__(kThreads)
 dispatch_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ x,
                        uint16_t *__restrict__ recv, int64_t T, int K, int64_t H, int64_t nrows,
                        int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -125,6 +152,7 @@ __global__ void __launch_bounds__(kThreads)
 combine_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ y,
                    const float *__restrict__ gates, uint4 *__restrict__ out, int64_t T, int K,
                    int64_t nvec, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -181,6 +209,7 @@ __global__ void __launch_bounds__(kThreads)
 combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ y,
                      const float *__restrict__ gates, uint4 *__restrict__ out, int64_t T, int K,
                      int64_t nvec, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -237,6 +266,7 @@ __global__ void __launch_bounds__(kThreads)
 combine_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *__restrict__ y,
                       const float *__restrict__ gates, uint16_t *__restrict__ out, int64_t T, int K,
                       int64_t H, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -266,6 +296,7 @@ combine_bwd_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restr
                        const uint4 *__restrict__ y, const float *__restrict__ gates,
                        uint4 *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
                        int64_t nvec, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -328,6 +359,7 @@ combine_bwd_split_kernel(const int32_t *__restrict__ slot_of, const uint4 *__res
                          const uint4 *__restrict__ y, const float *__restrict__ gates,
                          uint4 *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
                          int64_t nvec, int64_t nrows, int32_t *status) {
+  pdl_wait();
   __shared__ float red[kWarpsPerBlock][KMAX];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int half = wib & 1;
@@ -410,6 +442,7 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
                           const uint16_t *__restrict__ y, const float *__restrict__ gates,
                           uint16_t *__restrict__ dy, float *__restrict__ dgates, int64_t T, int K,
                           int64_t H, int64_t nrows, int32_t *status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -448,6 +481,7 @@ reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__
                        const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
                        const uint4 *__restrict__ rep, uint4 *__restrict__ home, int64_t nvec,
                        int R, int E, int B, int PMAX, int32_t *status) {
+  pdl_wait();
   int64_t n_exp = scalars[S_N_REPLICATED];
   if (n_exp < 0 || n_exp > E) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
@@ -543,6 +577,7 @@ __global__ void __launch_bounds__(512)
 comm_place_kernel(const int32_t *__restrict__ slot_of, int32_t *__restrict__ comm_index,
                   int32_t *__restrict__ counters, int64_t T, int K, int R, int64_t NvS,
                   int32_t *status) {
+  pdl_wait();
   extern __shared__ int cs[];  // [R] local counts, then [R] global bases
   int *cnt = cs, *base = cs + R;
   for (int d = threadIdx.x; d < R; d += blockDim.x) cnt[d] = 0;
@@ -587,6 +622,7 @@ __global__ void __launch_bounds__(kThreads)
 permute_rows_kernel(const int32_t *__restrict__ src_index, const int32_t *__restrict__ dst_index,
                     const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t npairs,
                     int64_t nvec, int64_t nrows) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -622,6 +658,7 @@ prefetch_weight_vec_kernel(const int32_t *__restrict__ replicated, const int32_t
                            const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
                            const uint4 *__restrict__ w, uint4 *__restrict__ rep_w, int64_t nvec,
                            int R, int E, int B, int PMAX, int32_t *status) {
+  pdl_wait();
   int64_t n_exp = scalars[S_N_REPLICATED];
   if (n_exp < 0 || n_exp > E) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
@@ -670,6 +707,7 @@ prefetch_weight_scalar_kernel(const int32_t *__restrict__ replicated, const int3
                               const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
                               const uint16_t *__restrict__ w, uint16_t *__restrict__ rep_w, int64_t W,
                               int R, int E, int B, int PMAX, int32_t *status) {
+  pdl_wait();
   int64_t n_exp = scalars[S_N_REPLICATED];
   if (n_exp < 0 || n_exp > E) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
@@ -704,6 +742,7 @@ reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t 
                           const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
                           const uint16_t *__restrict__ rep, uint16_t *__restrict__ home, int64_t P,
                           int R, int E, int B, int PMAX, int32_t *status) {
+  pdl_wait();
   int64_t n_exp = scalars[S_N_REPLICATED];
   if (n_exp < 0 || n_exp > E) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
@@ -774,12 +813,12 @@ extern "C" moonep_status_t moonep_dispatch(const moonep_config_t *cfg, const voi
   const int64_t nrows = d.R * d.NvS;
   if (d.H % 8 == 0 && aligned16(x) && aligned16(recv)) {
     const RowChunks rc = row_chunks<kDispatchU>(d.H / 8);
-    dispatch_chunk_kernel<kDispatchU><<<token_grid(T * rc.nch), kThreads, 0, st>>>(
+    launch(dispatch_chunk_kernel<kDispatchU>, token_grid(T * rc.nch), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(recv), T,
         (int)d.K, d.H / 8, rc.nch, rc.cl, nrows, dev_status);
   } else {
-    dispatch_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], x, recv, T, (int)d.K,
-                                                               d.H, nrows, dev_status);
+    launch(dispatch_scalar_kernel, token_grid(T), kThreads, 0, st, P.f[F_SLOT_OF], x, recv, T, (int)d.K,
+        d.H, nrows, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
@@ -796,16 +835,16 @@ extern "C" moonep_status_t moonep_combine(const moonep_config_t *cfg, const void
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS;
   if (d.H % 8 == 0 && aligned16(y) && aligned16(out) && d.K <= 8) {
-    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
         T, (int)d.K, d.H / 8, nrows, dev_status);
   } else if (d.H % 8 == 0 && aligned16(y) && aligned16(out)) {
-    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+    launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
         T, (int)d.K, d.H / 8, nrows, dev_status);
   } else {
-    combine_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], y, gates, out, T,
-                                                              (int)d.K, d.H, nrows, dev_status);
+    launch(combine_scalar_kernel, token_grid(T), kThreads, 0, st, P.f[F_SLOT_OF], y, gates, out, T,
+        (int)d.K, d.H, nrows, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
@@ -827,15 +866,15 @@ extern "C" moonep_status_t moonep_combine_backward(const moonep_config_t *cfg,
   const bool vec = d.H % 8 == 0 && aligned16(dout) && aligned16(y) && aligned16(dy);
   if (vec && d.K <= 8) {
     // two warps per token measured 6.5 TB/s against 6.1 for one
-    combine_bwd_split_kernel<2, 8><<<token_grid(2 * T), kThreads, 0, st>>>(
+    launch((combine_bwd_split_kernel<2, 8>), token_grid(2 * T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(dout), reinterpret_cast<const uint4 *>(y),
         gates, reinterpret_cast<uint4 *>(dy), dgates, T, (int)d.K, d.H / 8, nrows, dev_status);
   } else if (vec) {
-    combine_bwd_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+    launch(combine_bwd_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(dout), reinterpret_cast<const uint4 *>(y),
         gates, reinterpret_cast<uint4 *>(dy), dgates, T, (int)d.K, d.H / 8, nrows, dev_status);
   } else {
-    combine_bwd_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(
+    launch(combine_bwd_scalar_kernel, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], dout, y, gates, dy, dgates, T, (int)d.K, d.H, nrows, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
@@ -855,13 +894,13 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
   cudaStream_t st = to_cuda(stream);
   const unsigned grid = (unsigned)num_sms() * 8;
   if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
-    reduce_grad_vec_kernel<4, 4><<<grid, kThreads, 0, st>>>(
+    launch((reduce_grad_vec_kernel<4, 4>), grid, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(rep_grads),
         reinterpret_cast<uint4 *>(home_grads), P_elems / 8, (int)d.R, (int)d.E, (int)d.B,
         (int)d.PMAX, dev_status);
   } else {
-    reduce_grad_scalar_kernel<<<grid, kThreads, 0, st>>>(
+    launch(reduce_grad_scalar_kernel, grid, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], rep_grads, home_grads, P_elems, (int)d.R,
         (int)d.E, (int)d.B, (int)d.PMAX, dev_status);
@@ -883,16 +922,16 @@ extern "C" moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
   const int64_t nrows = d.R * d.NvS;
   // the combine kernels with unit weights: fmaf(1, y, acc) rounds like acc + y
   if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx) && d.K <= 8) {
-    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
         reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, nrows, dev_status);
   } else if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx)) {
-    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+    launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
         reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, nrows, dev_status);
   } else {
-    combine_scalar_kernel<<<token_grid(T), kThreads, 0, st>>>(P.f[F_SLOT_OF], d_recv, nullptr, dx,
-                                                              T, (int)d.K, d.H, nrows, dev_status);
+    launch(combine_scalar_kernel, token_grid(T), kThreads, 0, st, P.f[F_SLOT_OF], d_recv, nullptr, dx,
+        T, (int)d.K, d.H, nrows, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
@@ -911,13 +950,13 @@ extern "C" moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
   if (W % 8 == 0 && aligned16(weights) && aligned16(rep_weights)) {
     // many small blocks: the block scheduler balances the expert-major units
     const unsigned grid = (unsigned)num_sms() * 64;
-    prefetch_weight_vec_kernel<8><<<grid, kThreads, 0, st>>>(
+    launch(prefetch_weight_vec_kernel<8>, grid, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(weights),
         reinterpret_cast<uint4 *>(rep_weights), W / 8, (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX,
         dev_status);
   } else {
-    prefetch_weight_scalar_kernel<<<(unsigned)num_sms() * 8, kThreads, 0, st>>>(
+    launch(prefetch_weight_scalar_kernel, (unsigned)num_sms() * 8, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], weights, rep_weights, W, (int)d.R, (int)d.E,
         (int)d.B, (int)d.PMAX, dev_status);
@@ -952,16 +991,16 @@ extern "C" moonep_status_t moonep_dispatch_via_buffer(const moonep_config_t *cfg
   int32_t *counters = comm_index + N;
   if (cudaMemsetAsync(counters, 0, sizeof(int32_t) * d.R, st) != cudaSuccess) return MOONEP_ERR_CUDA;
   const unsigned blocks = (unsigned)((T + kCommTokensPerBlock - 1) / kCommTokensPerBlock);
-  comm_place_kernel<<<blocks, 512, 2 * d.R * sizeof(int), st>>>(P.f[F_SLOT_OF], comm_index, counters,
-                                                                 T, (int)d.K, (int)d.R, d.NvS,
-                                                                 dev_status);
+  launch(comm_place_kernel, blocks, 512, 2 * d.R * sizeof(int), st, P.f[F_SLOT_OF], comm_index, counters,
+      T, (int)d.K, (int)d.R, d.NvS,
+      dev_status);
   // the sender writes rows into the receivers' communication buffers
   const RowChunks rc = row_chunks<kDispatchU>(d.H / 8);
-  dispatch_chunk_kernel<kDispatchU><<<token_grid(T * rc.nch), kThreads, 0, st>>>(
+  launch(dispatch_chunk_kernel<kDispatchU>, token_grid(T * rc.nch), kThreads, 0, st,
       comm_index, reinterpret_cast<const uint4 *>(x), reinterpret_cast<uint4 *>(comm), T, (int)d.K,
       d.H / 8, rc.nch, rc.cl, nrows, dev_status);
   // the receiver permutes them into expert order
-  permute_rows_kernel<<<pair_grid(N), kThreads, 0, st>>>(
+  launch(permute_rows_kernel, pair_grid(N), kThreads, 0, st,
       comm_index, P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(comm),
       reinterpret_cast<uint4 *>(recv), N, d.H / 8, nrows);
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
@@ -984,16 +1023,16 @@ extern "C" moonep_status_t moonep_combine_via_buffer(const moonep_config_t *cfg,
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS, N = T * d.K;
   // the expert ranks permute their outputs back into arrival order
-  permute_rows_kernel<<<pair_grid(N), kThreads, 0, st>>>(
+  launch(permute_rows_kernel, pair_grid(N), kThreads, 0, st,
       P.f[F_SLOT_OF], comm_index, reinterpret_cast<const uint4 *>(y), reinterpret_cast<uint4 *>(comm),
       N, d.H / 8, nrows);
   // and the source ranks combine from the communication buffer
   if (d.K <= 8)
-    combine_vec_k_kernel<2, 8><<<token_grid(T), kThreads, 0, st>>>(
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
         comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
         (int)d.K, d.H / 8, nrows, dev_status);
   else
-    combine_vec_kernel<4><<<token_grid(T), kThreads, 0, st>>>(
+    launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
         (int)d.K, d.H / 8, nrows, dev_status);
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
