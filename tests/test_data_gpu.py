@@ -245,6 +245,29 @@ def test_reduce_grad_expert_with_many_pieces():
     assert (got == ref).mean() >= 0.999
 
 
+@pytest.mark.parametrize("R,P", [(80, 10000), (80, 8), (80, 13)])
+def test_reduce_grad_more_local_pieces_than_the_cache(R, P):
+    """All tokens on expert 0 across 80 ranks: 79 local pieces of one expert.
+
+    More pieces than the reduce kernel keeps in shared memory (64), so its
+    producer walks the piece tables again for the rest; P = 10000 makes rows
+    of three chunks with a ragged last one, P = 8 a single 16-byte chunk, and
+    P = 13 takes the unaligned path."""
+    E, K, S, B = R, 1, 8, 1
+    cfg, ocfg = configs(R, E, K, S, H=8, budget=B)
+    idx = np.zeros((R, S, K), np.int32)
+    ost, ot = oracle.plan(ocfg, idx)
+    gst, arena, gv, _ = gpu_plan(cfg, idx)
+    assert int(ot["n_piece"][0]) == R - 1 and int(ot["n_remote"][0]) == 0
+    rep = normal_bf16((R, B, P), seed=17, stream=11)
+    home = normal_bf16((E, P), seed=17, stream=12)
+    got = _reduce(cfg, arena, rep, home, P)
+    ref = oracle.reduce_grad(ocfg, ot, rep, home)
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999
+    assert np.array_equal(got[1:], home[1:])  # experts without replicas untouched
+
+
 def _dispatch_bwd(cfg, arena, drecv_np):
     import torch
     import token_dispatch_moonep_b200 as me

@@ -470,96 +470,253 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
 }
 
 // ----------------------------------------------------------- reduce_grad ---
-// Work units: (replicated expert, warp-chunk of 32*U column vectors).  Each
-// unit reads the home vectors, then the expert's pieces in plan order in groups
-// of G: the group's local replica vectors are all loaded before they are added,
-// so a warp keeps (G + 1) * U loads in flight; adds stay in ascending piece order.
-template <int U, int G>
-__global__ void __launch_bounds__(kThreads)
-reduce_grad_vec_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
-                       const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
-                       const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
-                       const uint4 *__restrict__ rep, uint4 *__restrict__ home, int64_t nvec,
-                       int R, int E, int B, int PMAX, int32_t *status) {
+// A shared-memory pipeline fed by bulk asynchronous copies.  Work units are
+// (replicated expert, 8 KB chunk of its row); a unit is one or more stages:
+// the first holds the home chunk and the expert's first two local replica
+// chunks, each further stage the next two.  One producer thread per CTA
+// issues cp.async.bulk copies (completion counted in bytes on the stage's
+// mbarrier); eight consumer warps add the stage's rows in fp32 in piece order
+// and, after the unit's last stage, store the bf16 result over the home chunk.
+// Four stages per CTA and two CTAs per SM keep ~150 KB per SM in flight with
+// no registers held for it.  Every wait is bounded; a wait that gives up sets
+// MOONEP_DEV_TIMEOUT, and the producer waits (bounded) for its copies before
+// the CTA exits.
+namespace rg {
+constexpr int kChunk = 8192;             // bytes of a row per unit
+constexpr int kSlots = 3;                // chunks per stage
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 8;
+constexpr int kThreadsRg = (kConsumerWarps + 1) * 32;
+constexpr int kSmem = kStages * kSlots * kChunk;
+constexpr int kPieceCache = 64;          // local pieces of one expert kept in shared memory
+constexpr int kVecPerLane = kChunk / 16 / (kConsumerWarps * 32);
+constexpr long long kWaitNs = 200LL * 1000 * 1000;
+static_assert(kVecPerLane * 16 * kConsumerWarps * 32 == kChunk, "chunk split over consumer lanes");
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+// true once the phase of the given parity has completed; false after kWaitNs
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (!mbar_test(bar, parity))
+    if ((long long)(now_ns() - t0) > kWaitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+struct Tables {
+  const int32_t *replicated, *scalars, *pbeg, *pend, *prank, *pwslot;
+  int R, E, B, PMAX;
+};
+
+// Expert of replicated entry i and its piece range; false if the tables are inconsistent.
+__device__ __forceinline__ bool expert_of(const Tables &t, int64_t i, int *e, int *b, int *en) {
+  *e = t.replicated[i];
+  if (*e < 0 || *e >= t.E) return false;
+  *b = t.pbeg[*e];
+  *en = t.pend[*e];
+  return *b >= 0 && *en <= t.PMAX && *en >= *b;
+}
+__device__ __forceinline__ bool local_piece(const Tables &t, int pc, int *row) {
+  const int ws = t.pwslot[pc], rk = t.prank[pc];
+  *row = rk * t.B + ws;
+  return ws >= 0 && ws < t.B && rk >= 0 && rk < t.R;
+}
+}  // namespace rg
+
+__global__ void __launch_bounds__(rg::kThreadsRg, 1)
+reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__restrict__ home,
+                        int64_t nvec, int32_t *status) {
+  using namespace rg;
   pdl_wait();
-  int64_t n_exp = scalars[S_N_REPLICATED];
-  if (n_exp < 0 || n_exp > E) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  __shared__ int pcache[kPieceCache];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int64_t n_exp = t.scalars[S_N_REPLICATED];
+  if (n_exp < 0 || n_exp > t.E) {
+    if (blockIdx.x == 0 && tid == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
     n_exp = 0;
   }
-  const int64_t per_exp = (nvec + 32 * U - 1) / (32 * U);  // warp-chunks per expert
-  const int64_t total = n_exp * per_exp;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
-  for (int64_t w = warp_g; w < total; w += nwarps) {
-    const int e = replicated[w / per_exp];
-    const int64_t v0 = (w % per_exp) * 32 * U;
-    const int b = e >= 0 && e < E ? pbeg[e] : 0, en = e >= 0 && e < E ? pend[e] : -1;
-    if (e < 0 || e >= E || b < 0 || en > PMAX || en < b) {
-      if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
-      continue;
+  const int64_t rowbytes = nvec * 16;
+  const int64_t nch = (rowbytes + kChunk - 1) / kChunk;
+  const int64_t total = n_exp * nch;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
     }
-    uint4 *hrow = home + (int64_t)e * nvec;
-    float acc[U][8];
-#pragma unroll
-    for (int u = 0; u < U; u++) {
-      const int64_t v = v0 + u * 32 + lane;
-      const uint4 q = v < nvec ? hrow[v] : make_uint4(0, 0, 0, 0);
-      const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        acc[u][2 * i] = bf16_lo(wd[i]);
-        acc[u][2 * i + 1] = bf16_hi(wd[i]);
-      }
-    }
-    for (int pc0 = b; pc0 < en; pc0 += G) {
-      uint4 q[G][U];
-      bool use[G];
-#pragma unroll
-      for (int g = 0; g < G; g++) {
-        const int pc = pc0 + g;
-        const int ws = pc < en ? pwslot[pc] : -1;
-        const int rk = pc < en ? prank[pc] : -1;
-        use[g] = ws >= 0;
-        if (use[g] && (ws >= B || rk < 0 || rk >= R)) {
-          if (lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
-          use[g] = false;
-        }
-        const uint4 *rrow = rep + ((int64_t)(use[g] ? rk : 0) * B + (use[g] ? ws : 0)) * nvec;
-#pragma unroll
-        for (int u = 0; u < U; u++) {
-          const int64_t v = v0 + u * 32 + lane;
-          q[g][u] = (use[g] && v < nvec) ? __ldcs(rrow + v) : make_uint4(0, 0, 0, 0);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // Both roles walk the same sequence: units u = blockIdx.x + j * gridDim.x,
+  // each split into ng = max(1, ceil(local pieces / 2)) stages, stage k of the
+  // sequence in buffer k % kStages.
+  if (warp == kConsumerWarps) {  // ------------------------------- producer
+    if (lane != 0) return;
+    int64_t k = 0, cur = -1;
+    int e = 0, b = 0, en = 0, nl = 0;
+    bool good = false, ok = true;
+    for (int64_t u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      const int64_t i = u / nch;
+      if (i != cur) {  // a new expert: list its local pieces once
+        cur = i;
+        good = expert_of(t, i, &e, &b, &en);
+        nl = 0;
+        for (int pc = b; good && pc < en; pc++) {
+          int row;
+          if (!local_piece(t, pc, &row)) continue;
+          if (nl < kPieceCache) pcache[nl] = row;
+          nl++;
         }
       }
+      if (!good) continue;
+      const int64_t off = (u % nch) * kChunk;
+      const uint32_t bytes = (uint32_t)(rowbytes - off < kChunk ? rowbytes - off : kChunk);
+      const int ng = nl > 0 ? (nl + 1) / 2 : 1;
+      int li = 0, pc = b;
+      for (int g = 0; g < ng; g++, k++) {
+        const int s = (int)(k % kStages);
+        if (!mbar_wait(&empty[s], (uint32_t)((k / kStages) & 1) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        const uint8_t *src[kSlots];
+        int ns = 0;
+        if (g == 0) src[ns++] = reinterpret_cast<const uint8_t *>(home + (int64_t)e * nvec) + off;
+        while (ns < (g == 0 ? kSlots : kSlots - 1) && li < nl) {
+          int row = 0;
+          if (nl <= kPieceCache) {
+            row = pcache[li];
+          } else {  // more local pieces than the cache holds: walk the tables again
+            while (pc < en && !local_piece(t, pc, &row)) pc++;
+            pc++;
+          }
+          li++;
+          src[ns++] = reinterpret_cast<const uint8_t *>(rep + (int64_t)row * nvec) + off;
+        }
+        mbar_expect_tx(&full[s], bytes * (uint32_t)ns);
+        uint8_t *dst = stage_mem + (size_t)s * kSlots * kChunk;
+        for (int q = 0; q < ns; q++) bulk_load(dst + (size_t)q * kChunk, src[q], bytes, &full[s]);
+      }
+    }
+    if (!ok) set_status(status, MOONEP_DEV_TIMEOUT);
+    for (int64_t j = k > kStages ? k - kStages : 0; j < k; j++)  // copies land before exit
+      mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  int64_t k = 0, cur = -1;
+  int e = 0, nl = 0;
+  bool good = false, ok = true;
+  for (int64_t u = blockIdx.x; u < total && ok; u += gridDim.x) {
+    const int64_t i = u / nch;
+    if (i != cur) {
+      cur = i;
+      int b = 0, en = 0;
+      good = expert_of(t, i, &e, &b, &en);
+      nl = 0;
+      for (int pc = b; good && pc < en; pc++) {
+        int row;
+        nl += local_piece(t, pc, &row) ? 1 : 0;
+      }
+      if (!good && warp == 0 && lane == 0) set_status(status, MOONEP_DEV_BAD_PLAN);
+    }
+    if (!good) continue;
+    const int64_t off = (u % nch) * kChunk;
+    const int64_t nv = (rowbytes - off < kChunk ? rowbytes - off : kChunk) / 16;
+    const int ng = nl > 0 ? (nl + 1) / 2 : 1;
+    float acc[kVecPerLane][8];
+    int left = nl;
+    for (int g = 0; g < ng; g++, k++) {
+      const int s = (int)(k % kStages);
+      if (!mbar_wait(&full[s], (uint32_t)((k / kStages) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint4 *slot = reinterpret_cast<const uint4 *>(stage_mem + (size_t)s * kSlots * kChunk);
+      int q = 0;
+      if (g == 0) {  // the home chunk starts the sum
 #pragma unroll
-      for (int g = 0; g < G; g++) {
-        if (!use[g]) continue;
+        for (int j = 0; j < kVecPerLane; j++) {
+          const int64_t v = (warp * kVecPerLane + j) * 32 + lane;
+          const uint4 h = v < nv ? slot[v] : make_uint4(0, 0, 0, 0);
+          const uint32_t wd[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
-        for (int u = 0; u < U; u++) {
-          const uint32_t wd[4] = {q[g][u].x, q[g][u].y, q[g][u].z, q[g][u].w};
+          for (int w = 0; w < 4; w++) {
+            acc[j][2 * w] = bf16_lo(wd[w]);
+            acc[j][2 * w + 1] = bf16_hi(wd[w]);
+          }
+        }
+        q = 1;
+      }
+      const int np = left < kSlots - 1 ? left : kSlots - 1;
+      left -= np;
+      for (int pq = 0; pq < np; pq++, q++) {  // replicas in piece order
+        const uint4 *sl = slot + (int64_t)q * (kChunk / 16);
 #pragma unroll
-          for (int i = 0; i < 4; i++) {
-            acc[u][2 * i] = __fadd_rn(acc[u][2 * i], bf16_lo(wd[i]));
-            acc[u][2 * i + 1] = __fadd_rn(acc[u][2 * i + 1], bf16_hi(wd[i]));
+        for (int j = 0; j < kVecPerLane; j++) {
+          const int64_t v = (warp * kVecPerLane + j) * 32 + lane;
+          const uint4 r = v < nv ? sl[v] : make_uint4(0, 0, 0, 0);
+          const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int w = 0; w < 4; w++) {
+            acc[j][2 * w] = __fadd_rn(acc[j][2 * w], bf16_lo(wd[w]));
+            acc[j][2 * w + 1] = __fadd_rn(acc[j][2 * w + 1], bf16_hi(wd[w]));
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
+    if (!ok) break;
+    uint4 *hrow = home + (int64_t)e * nvec + off / 16;
 #pragma unroll
-    for (int u = 0; u < U; u++) {
-      const int64_t v = v0 + u * 32 + lane;
-      if (v < nvec) {
+    for (int j = 0; j < kVecPerLane; j++) {
+      const int64_t v = (warp * kVecPerLane + j) * 32 + lane;
+      if (v < nv) {
         uint4 o;
-        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        o.x = pack_bf16x2(acc[j][0], acc[j][1]);
+        o.y = pack_bf16x2(acc[j][2], acc[j][3]);
+        o.z = pack_bf16x2(acc[j][4], acc[j][5]);
+        o.w = pack_bf16x2(acc[j][6], acc[j][7]);
         hrow[v] = o;
       }
     }
   }
+  if (!ok && lane == 0) set_status(status, MOONEP_DEV_TIMEOUT);
 }
 
 // ------------------------------------------------ copy-through-buffer mode ---
@@ -892,15 +1049,24 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
   if (d.B == 0) return MOONEP_OK;  // no replica slots, nothing to fold
   PlanPtrs P = plan_ptrs(d, plan_arena);
   cudaStream_t st = to_cuda(stream);
-  const unsigned grid = (unsigned)num_sms() * 8;
   if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
-    launch((reduce_grad_vec_kernel<4, 4>), grid, kThreads, 0, st,
-        P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
-        P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], reinterpret_cast<const uint4 *>(rep_grads),
-        reinterpret_cast<uint4 *>(home_grads), P_elems / 8, (int)d.R, (int)d.E, (int)d.B,
-        (int)d.PMAX, dev_status);
+    // bulk copies need 16-byte aligned rows: P % 8 == 0 and aligned bases
+    if (cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             rg::kSmem) != cudaSuccess)
+      return MOONEP_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_grad_bulk_kernel,
+                                                      rg::kThreadsRg, rg::kSmem) != cudaSuccess ||
+        per_sm < 1)
+      return MOONEP_ERR_CUDA;
+    const rg::Tables t{P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN],
+                       P.f[F_EXP_PIECE_END], P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT],
+                       (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX};
+    launch(reduce_grad_bulk_kernel, (unsigned)(num_sms() * per_sm), rg::kThreadsRg, rg::kSmem, st,
+        t, reinterpret_cast<const uint4 *>(rep_grads), reinterpret_cast<uint4 *>(home_grads),
+        P_elems / 8, dev_status);
   } else {
-    launch(reduce_grad_scalar_kernel, grid, kThreads, 0, st,
+    launch(reduce_grad_scalar_kernel, (unsigned)num_sms() * 8, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], rep_grads, home_grads, P_elems, (int)d.R,
         (int)d.E, (int)d.B, (int)d.PMAX, dev_status);
