@@ -34,6 +34,7 @@ namespace {
 // process-wide diagnostics (moonep_debug_set_wait)
 std::atomic<long long> g_wait_limit_ns{200LL * 1000 * 1000};
 std::atomic<int> g_phantom_arrivals{0};
+std::atomic<bool> g_plan_pdl{true};
 
 constexpr int kStBad = 1, kStCapacity = 2, kStTimeout = 8;
 // Odd step between launch epochs: values left in a reused workspace (previous
@@ -610,6 +611,10 @@ __device__ __forceinline__ bool wait_flag(const int32_t *flag, int v, long long 
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  // launched with programmatic stream serialisation: wait here until the
+  // kernel before it in the stream (the router's top-k, the previous layer)
+  // has completed and its writes are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) int smem[];
   __shared__ int s_epoch, s_state, s_ok;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -923,16 +928,24 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   lc.blockDim = dim3(kPlanThreads);
   lc.dynamicSmemBytes = smem;
   lc.stream = to_cuda(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
-  lc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&lc, plan_kernel, a) != cudaSuccess) {
+  // programmatic dependent launch hides the launch gap after the previous
+  // kernel; without it (a runtime that refuses the pair) the launch is plain
+  lc.numAttrs = g_plan_pdl.load(std::memory_order_relaxed) ? 2 : 1;
+  if (cudaLaunchKernelEx(&lc, plan_kernel, a) == cudaSuccess) return MOONEP_OK;
+  cudaGetLastError();
+  if (lc.numAttrs == 2) {
+    g_plan_pdl.store(false);
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, plan_kernel, a) == cudaSuccess) return MOONEP_OK;
     cudaGetLastError();
-    return MOONEP_ERR_CUDA;
   }
-  return MOONEP_OK;
+  return MOONEP_ERR_CUDA;
 }
 
 extern "C" moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals) {
