@@ -223,7 +223,11 @@ MOONEP_API moonep_status_t moonep_combine_backward(const moonep_config_t *cfg, c
  *     home[e, :] = bf16( float(home[e, :]) + sum_d float(rep[d, wslot_d(e), :]) )
  * in fp32, in place.  rep_grads device bf16 [R, budget, P]; home_grads device
  * bf16 [E, P]; P >= 1 elements per expert gradient.  Remote pieces have no
- * replica slot and contribute nothing (TRAIN plans flag them as BUDGET). */
+ * replica slot and contribute nothing (TRAIN plans flag them as BUDGET).
+ * With P % 8 == 0 and 16-byte aligned buffers the kernel stages rows in shared
+ * memory with bulk asynchronous copies; its internal waits are bounded and one
+ * that gives up (not possible with a consistent plan) sets MOONEP_DEV_TIMEOUT.
+ * dev_status bits: BAD_PLAN (inconsistent plan tables), TIMEOUT. */
 MOONEP_API moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
                                    const uint16_t *rep_grads, uint16_t *home_grads, int64_t P,
                                    int32_t *dev_status, moonep_stream_t stream);
