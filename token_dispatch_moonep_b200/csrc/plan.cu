@@ -230,9 +230,7 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
   for (int j = 0; j < kPairsPerThread; j++) {
     if (j >= ppt) break;  // uniform across the block
     const int e = ev[j];
-    uint32_t peers = 0;
-#pragma unroll
-    for (int l = 0; l < 32; l++) peers |= (uint32_t)(__shfl_sync(0xffffffffu, e, l) == e) << l;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);  // lanes holding the same id
     const int prev = e >= 0 ? myh[e] : 0;
     const int r = __popc(peers & lt);
     rk[j] = prev + r;
@@ -286,6 +284,81 @@ __device__ __forceinline__ SolveSmem carve(const Dims &d, int *s) {
 
 __host__ __device__ inline size_t solve_smem_ints(const Dims &d) {
   return 10 * d.E + 11 * d.R + 5 * d.PMAX + 4 * 33 + 8 + 4 + 4 * kPlanThreads;
+}
+
+// Solver side of the arrivals when every worker has one chunk: warp w waits
+// for chunks w, w + 16, ... (and the phantom arrivals of the timeout test) and
+// adds each chunk's histogram into its own partial row part[w][E] as soon as
+// the chunk's flag shows this launch's epoch, so most of the summing overlaps
+// the wait.  Then cnt[e] = sum of the 16 partials.  part may alias cnt (each
+// column is reduced by one thread).  Returns kStTimeout / kStBad bits.
+__device__ int gather_counts(const PlanArgs &a, int epoch, int *part, int *cnt, int *flags) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = (int)a.d.E;
+  const int64_t ntot = a.nc + a.phantom;
+  if (tid == 0) flags[0] = 0;
+  for (int e = lane; e < E; e += 32) part[warp * E + e] = 0;
+  __syncthreads();
+  int st = 0;
+  const unsigned long long t0 = now_ns();
+  for (int64_t c0 = warp; c0 < ntot && st == 0; c0 += (int64_t)kPlanWarps * 32) {
+    const int64_t c = c0 + (int64_t)kPlanWarps * lane;  // this lane's chunk in the batch
+    bool pend = c < ntot;
+    unsigned pending = __ballot_sync(0xffffffffu, pend);
+    while (pending) {
+      const bool arrived = pend && ld_relaxed(a.arrive + c) == epoch;
+      unsigned got = __ballot_sync(0xffffffffu, arrived);
+      if (!got) {
+        if ((long long)(now_ns() - t0) > a.wait_ns) {
+          st = kStTimeout;
+          break;
+        }
+        __nanosleep(32);
+        continue;
+      }
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+      pending &= ~got;
+      if (arrived) pend = false;
+      bool bad = arrived && c < a.nc && __ldcg(a.badmark + c) == epoch;
+      if (__any_sync(0xffffffffu, bad)) st |= kStBad;
+      while (got) {  // add up to four arrived chunks per pass, their loads in flight together
+        int64_t cj[4];
+        int n = 0;
+        while (got && n < 4) {
+          const int j = __ffs(got) - 1;
+          got &= got - 1;
+          const int64_t cc = c0 + (int64_t)kPlanWarps * j;
+          if (cc < a.nc) cj[n++] = cc;
+        }
+        for (int qb = 0; qb < E; qb += 32 * 8) {
+          int v[4][8];
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+#pragma unroll
+            for (int q = 0; q < 8; q++) {
+              const int col = qb + q * 32 + lane;
+              v[i][q] = (i < n && col < E) ? __ldcg(a.hist + cj[i] * E + col) : 0;
+            }
+#pragma unroll
+          for (int q = 0; q < 8; q++) {
+            const int col = qb + q * 32 + lane;
+            if (col < E) part[warp * E + col] += v[0][q] + v[1][q] + v[2][q] + v[3][q];
+          }
+        }
+      }
+    }
+  }
+  if (lane == 0 && st) atomicOr(flags, st);
+  __syncthreads();
+  st = flags[0];
+  for (int e = tid; e < E; e += kPlanThreads) {
+    int sum = 0;
+#pragma unroll
+    for (int w = 0; w < kPlanWarps; w++) sum += part[w * E + e];
+    cnt[e] = sum;
+  }
+  __syncthreads();
+  return st;
 }
 
 // Per-expert exclusive scan of the histograms over chunks, in place (the
@@ -623,29 +696,34 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   int32_t *gen = a.sync + kSyncGen, *done = a.sync + kSyncDone;
   int32_t *state_w = a.sync + kSyncState, *tables = a.sync + kSyncTables;
 
-  if (tid == 0) s_epoch = (int)((unsigned)*((volatile int32_t *)gen) + kEpochStep);
-  __syncthreads();
-  const int epoch = s_epoch;
+  // the generation word: workers need it only when they publish, so its load
+  // overlaps their counting
+  int gen_v = 0;
+  if (tid == 0) gen_v = *((volatile int32_t *)gen);
 
   // ================================================================ solver ==
   if (blockIdx.x == 0) {
-    if (warp == 0) {
-      const bool ok = warp_wait_all(a.arrive, a.nc + a.phantom, epoch, a.wait_ns);
-      bool b = false;
-      for (int64_t c = lane; c < a.nc; c += 32) b |= __ldcg(a.badmark + c) == epoch;
-      b = __any_sync(0xffffffffu, b);
-      if (lane == 0) s_state = (ok ? 0 : kStTimeout) | (b ? kStBad : 0);
-      __threadfence();
-    }
+    if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
     __syncthreads();
-    int st = s_state;
-    if (tid == 0) *((volatile int32_t *)gen) = epoch;  // every CTA read it before arriving
+    const int epoch = s_epoch;
     SolveSmem m = carve(d, smem);
-    if (st == 0) {
-      if (a.nc > a.workers) chunk_bases(a, m.cnt);
-      else column_sums(a.hist, E, a.nc, m.cnt, m.red);
-      st = solve_core(a, m);
+    int st;
+    if (a.nc <= a.workers) {
+      st = gather_counts(a, epoch, smem, m.cnt, &s_state);
+    } else {
+      if (warp == 0) {
+        const bool ok = warp_wait_all(a.arrive, a.nc + a.phantom, epoch, a.wait_ns);
+        bool b = false;
+        for (int64_t c = lane; c < a.nc; c += 32) b |= __ldcg(a.badmark + c) == epoch;
+        b = __any_sync(0xffffffffu, b);
+        if (lane == 0) s_state = (ok ? 0 : kStTimeout) | (b ? kStBad : 0);
+      }
+      __syncthreads();
+      st = s_state;
+      if (st == 0) chunk_bases(a, m.cnt);
     }
+    if (tid == 0) *((volatile int32_t *)gen) = epoch;  // every CTA read it before arriving
+    if (st == 0) st = solve_core(a, m);
     if (tid == 0) {
       if (st & kStTimeout) set_status(a.status, MOONEP_DEV_TIMEOUT);
       if (st & kStCapacity) set_status(a.status, MOONEP_DEV_CAPACITY);
@@ -671,8 +749,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   const int wk = blockIdx.x - 1, W = a.workers;
   const bool single = a.nc <= W;  // at most one chunk per worker: ids and ranks stay in registers
   int ev[kPairsPerThread], rk[kPairsPerThread];
+  int epoch = 0;
+  bool have_epoch = false;
   for (int64_t k = wk; k < a.nc; k += W) {
     const bool bad = __syncthreads_or(count_chunk(a, k, smem, ev, rk));
+    if (!have_epoch) {
+      if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
+      __syncthreads();
+      epoch = s_epoch;
+      have_epoch = true;
+    }
     if (!single) {
       const int64_t base = k * a.ch + (int64_t)warp * 32 * a.ppt;
 #pragma unroll
@@ -686,6 +772,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       __threadfence();
       st_release(a.arrive + k, epoch);
     }
+  }
+  if (!have_epoch) {  // a worker without a chunk
+    if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
+    __syncthreads();
+    epoch = s_epoch;
   }
   int *tb = smem;  // placement tables, see place_chunk
   // base offsets of my chunk: sums of the histograms of the chunks before it
