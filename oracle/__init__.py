@@ -12,7 +12,7 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
   experts are duplicated onto other ranks within a per-rank replica-slot budget
   (same page, replica-slot paragraph), buffers have a fixed NvS = S*K +
   alignment padding rows ("MoonshotAI/MoonEP 딥다이브" §4 pattern 2).  The
-  tie-breaks are this build's fixed reading (see the C file header).  Pinned by:
+  tie-breaks are a fixed reading stated in the C file header.  Pinned by:
   a hand-derived worked example; closed-form degenerate routings (all tokens on
   one expert, already-balanced routing); invariants on random routings (S*K
   rows per rank, bijection pairs -> rows, row expert = routed expert, replica
