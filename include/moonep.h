@@ -176,12 +176,15 @@ MOONEP_API moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const 
                                               void *plan_arena, int32_t *dev_status,
                                               moonep_stream_t stream);
 
-/* Diagnostics for the plan kernel's bounded waits (process-wide, host-side).
+/* Diagnostics for the bounded in-kernel waits (process-wide, host-side).
  * The plan is one cooperative launch whose CTAs wait for each other twice;
- * each wait gives up after `limit_ns` nanoseconds (default 200 ms), sets
- * MOONEP_DEV_TIMEOUT and leaves an invalid plan (slot_of = -1) instead of
- * hanging.  `phantom_arrivals` (tests only, 0..32) makes the solving CTA also
- * wait for that many arrivals that no CTA ever makes, forcing the timeout. */
+ * reduce_grad's pipeline waits on shared-memory barriers for its bulk copies.
+ * Each wait gives up after `limit_ns` nanoseconds (default 200 ms) and sets
+ * MOONEP_DEV_TIMEOUT instead of hanging (a timed-out plan is invalid:
+ * slot_of = -1).  `phantom_arrivals` (tests only, 0..32) forces the timeout:
+ * the plan's solving CTA also waits for that many arrivals that no CTA ever
+ * makes, and each reduce_grad CTA's first stage expects 16 bytes per phantom
+ * arrival more than its copies deliver. */
 MOONEP_API moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals);
 
 /* Fill `out` with device pointers into `plan_arena` (pure host arithmetic). */

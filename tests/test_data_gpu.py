@@ -433,3 +433,29 @@ def test_chained_calls_without_host_syncs():
     close(to_np(home), ref_home)
     valid = ot2["slot_src"] >= 0
     close(to_np(recv)[valid], ref_recv2[valid])
+
+
+def test_reduce_grad_forced_timeout_reports_status_and_context_stays_usable():
+    """reduce_grad's pipeline waits are bounded: a stage that expects bytes no copy
+    delivers (the debug hook) ends the kernel with TIMEOUT instead of hanging, and
+    the next call on the same context is correct."""
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S, B, P = 8, 32, 4, 256, 4, 2048
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=6.0, seed=6, budget=B)
+    assert int(ot["n_piece"][0]) > 0
+    rep = normal_bf16((R, B, P), seed=6, stream=11)
+    home = normal_bf16((E, P), seed=6, stream=12)
+    import torch
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    h = to_dev(home)
+    try:
+        me.moonep_debug_set_wait(2_000_000, 1)  # 2 ms, 16 bytes that never arrive
+        me.moonep_reduce_grad(cfg, arena, to_dev(rep), h, P, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) & me.DEV_TIMEOUT
+    finally:
+        me.moonep_debug_set_wait(me.DEFAULT_WAIT_NS, 0)
+    got = _reduce(cfg, arena, rep, home, P)
+    ref = oracle.reduce_grad(ocfg, ot, rep, home)
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert (got == ref).mean() >= 0.999

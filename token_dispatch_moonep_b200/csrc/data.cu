@@ -479,9 +479,10 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
 // and, after the unit's last stage, store the bf16 result over the home chunk.
 // Three stages of four chunks per CTA and two CTAs per SM keep up to 192 KB
 // per SM in flight with no registers held for it (measured against 4 stages
-// of 3 chunks: equal at 10 pieces over 6 experts, 6% faster at 59 over 54).  Every wait is bounded; a wait that gives up sets
-// MOONEP_DEV_TIMEOUT, and the producer waits (bounded) for its copies before
-// the CTA exits.
+// of 3 chunks: equal at 10 pieces over 6 experts, 6% faster at 59 over 54).
+// Every wait is bounded (moonep_debug_set_wait's limit); a wait that gives up
+// sets MOONEP_DEV_TIMEOUT, and the producer waits (bounded) for its copies
+// before the CTA exits.
 namespace rg {
 constexpr int kChunk = 8192;             // bytes of a row per unit
 constexpr int kSlots = 4;                // chunks per stage
@@ -491,7 +492,6 @@ constexpr int kThreadsRg = (kConsumerWarps + 1) * 32;
 constexpr int kSmem = kStages * kSlots * kChunk;
 constexpr int kPieceCache = 64;          // local pieces of one expert kept in shared memory
 constexpr int kVecPerLane = kChunk / 16 / (kConsumerWarps * 32);
-constexpr long long kWaitNs = 200LL * 1000 * 1000;
 static_assert(kVecPerLane * 16 * kConsumerWarps * 32 == kChunk, "chunk split over consumer lanes");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -520,12 +520,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// true once the phase of the given parity has completed; false after kWaitNs
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// true once the phase of the given parity has completed; false after limit_ns
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
   while (!mbar_test(bar, parity))
-    if ((long long)(now_ns() - t0) > kWaitNs) return false;
+    if ((long long)(now_ns() - t0) > limit_ns) return false;
   return true;
 }
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -538,6 +538,8 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
 struct Tables {
   const int32_t *replicated, *scalars, *pbeg, *pend, *prank, *pwslot;
   int R, E, B, PMAX;
+  long long wait_ns;  // limit of every mbarrier wait
+  int phantom_tx;     // bytes the first stage expects beyond its copies (0; tests force a timeout)
 };
 
 // Expert of replicated entry i and its piece range; false if the tables are inconsistent.
@@ -614,7 +616,7 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
       int li = 0, pc = b;
       for (int g = 0; g < ng; g++, k++) {
         const int s = (int)(k % kStages);
-        if (!mbar_wait(&empty[s], (uint32_t)((k / kStages) & 1) ^ 1u)) {
+        if (!mbar_wait(&empty[s], (uint32_t)((k / kStages) & 1) ^ 1u, t.wait_ns)) {
           ok = false;
           break;
         }
@@ -632,14 +634,14 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
           li++;
           src[ns++] = reinterpret_cast<const uint8_t *>(rep + (int64_t)row * nvec) + off;
         }
-        mbar_expect_tx(&full[s], bytes * (uint32_t)ns);
+        mbar_expect_tx(&full[s], bytes * (uint32_t)ns + (k == 0 ? (uint32_t)t.phantom_tx : 0u));
         uint8_t *dst = stage_mem + (size_t)s * kSlots * kChunk;
         for (int q = 0; q < ns; q++) bulk_load(dst + (size_t)q * kChunk, src[q], bytes, &full[s]);
       }
     }
     if (!ok) set_status(status, MOONEP_DEV_TIMEOUT);
     for (int64_t j = k > kStages ? k - kStages : 0; j < k; j++)  // copies land before exit
-      mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1));
+      mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1), t.wait_ns);
     return;
   }
 
@@ -668,7 +670,7 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
     int left = nl;
     for (int g = 0; g < ng; g++, k++) {
       const int s = (int)(k % kStages);
-      if (!mbar_wait(&full[s], (uint32_t)((k / kStages) & 1))) {
+      if (!mbar_wait(&full[s], (uint32_t)((k / kStages) & 1), t.wait_ns)) {
         ok = false;
         break;
       }
@@ -1068,7 +1070,8 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
       return MOONEP_ERR_CUDA;
     const rg::Tables t{P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN],
                        P.f[F_EXP_PIECE_END], P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT],
-                       (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX};
+                       (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX, debug_wait_limit_ns(),
+                       debug_phantom() > 0 ? 16 * debug_phantom() : 0};
     launch(reduce_grad_bulk_kernel, (unsigned)(num_sms() * per_sm), rg::kThreadsRg, rg::kSmem, st,
         t, reinterpret_cast<const uint4 *>(rep_grads), reinterpret_cast<uint4 *>(home_grads),
         P_elems / 8, dev_status);

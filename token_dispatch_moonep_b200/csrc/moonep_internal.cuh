@@ -11,6 +11,12 @@
 
 namespace moonep {
 
+// Diagnostics set by moonep_debug_set_wait (process-wide, host side): the
+// time limit of every bounded in-kernel wait, and the phantom count that
+// forces a wait to run out (tests only).
+long long debug_wait_limit_ns();
+int debug_phantom();
+
 constexpr int kPlanThreads = 512;   // threads per CTA of the plan kernel
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kPairsPerThread = 16;  // most pairs per thread in one plan chunk

@@ -1039,6 +1039,11 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   return MOONEP_ERR_CUDA;
 }
 
+namespace moonep {
+long long debug_wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+int debug_phantom() { return g_phantom_arrivals.load(std::memory_order_relaxed); }
+}  // namespace moonep
+
 extern "C" moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals) {
   if (limit_ns < 0 || phantom_arrivals < 0 || phantom_arrivals > kSyncMaxPhantom)
     return MOONEP_ERR_INVALID_ARG;
