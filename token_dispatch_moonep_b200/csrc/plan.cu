@@ -737,10 +737,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       st_release(done, epoch);
     }
     if (st == 0) solve_outputs(a, m);
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      st_release(tables, epoch);
+    if (d.A > 1) {  // only the padding fill (A > 1) waits for the finished tables
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        st_release(tables, epoch);
+      }
     }
     return;
   }
