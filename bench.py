@@ -76,8 +76,9 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def ncu_traffic():
-    """Per-kernel DRAM bytes per launch from the committed ncu summary, if still current."""
+def ncu_traffic(workload, maxvio, seed):
+    """Per-kernel DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this workload (name, maxvio, seed) and the kernel's source has not changed since."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     out = {}
@@ -96,7 +97,9 @@ def ncu_traffic():
         if ln.startswith("#") or not ln.strip():
             continue
         parts = dict(kv.split("=", 1) for kv in ln.split())
-        if src_hash.get(parts.get("source")) == parts.get("sha"):
+        same_case = (parts.get("workload") == workload and parts.get("seed") == str(seed)
+                     and abs(float(parts.get("maxvio", "nan")) - maxvio) < 1e-9)
+        if same_case and src_hash.get(parts.get("source")) == parts.get("sha"):
             out[parts["kernel"]] = float(parts["bytes_per_launch"])
     return out
 
@@ -554,7 +557,7 @@ def main():
                       "frac": b[name] / (avg * 1e-3) / 1e9 / peak, "share": sum(ts) / per_total}
     kern["plan"].pop("frac")
     dom = max((k for k in kern if k != "plan"), key=lambda k: kern[k]["ms"])
-    traffic = ncu_traffic().get(dom)
+    traffic = ncu_traffic(w.name if args.scale_s <= 1 else None, mv, args.seed).get(dom)
     roof = {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["GBs"], "peak": peak,
             "unit": "GB/s", "frac": kern[dom]["GBs"] / peak, "traffic": traffic,
             "peak_source": f"{peak_src} copy bandwidth"}

@@ -53,6 +53,10 @@ def test_single_process_helpers():
     assert bench.whole_job_gbs(6.5e9, 1, 1.0) == pytest.approx(6500.0)
     b = bench.algorithmic_bytes(8, 4096, 8, 7168)
     assert b["dispatch"] == 4228907008 and b["combine"] == 4229955584
+    # captured DRAM traffic belongs to one workload: never reported for another
+    assert bench.ncu_traffic("ep8_e32_k4_s256_h512", 0.2, 0) == {}
+    assert bench.ncu_traffic("ep8_e256_k8_s4096_h7168", 20.0, 0) == {}
+    assert bench.ncu_traffic("ep8_e256_k8_s4096_h7168", 0.2, 1) == {}
 
 
 @pytest.mark.parametrize("rank", [0, 1])
