@@ -109,6 +109,19 @@ def test_bad_expert_id_sets_status_and_invalidates_plan():
     assert st & me.DEV_BAD_EXPERT_ID
 
 
+def test_bad_expert_id_in_the_first_chunk_of_a_large_plan():
+    """A bad id in chunk 0 of 128: every CTA still arrives before the solver moves
+    on, so the status is exactly BAD_EXPERT_ID (no timeout) and the plan is invalid."""
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S = 8, 64, 8, 2048
+    cfg, _ = configs(R, E, K, S)
+    idx, _, _ = make_routing(R, E, K, S, 3.0, seed=12)
+    idx[0, 0, 0] = E + 5
+    st, arena, gv, _ = gpu_plan(cfg, idx)
+    assert st == me.DEV_BAD_EXPERT_ID
+    assert (gv["slot_of"] == -1).all() and (gv["slot_src"] == -1).all()
+
+
 def test_budget_flag_only_in_training_mode():
     import token_dispatch_moonep_b200 as me
     idx = np.zeros((4, 10, 1), np.int32)  # expert 0 overflows onto 3 ranks

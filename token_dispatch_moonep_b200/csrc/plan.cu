@@ -301,7 +301,9 @@ __device__ int gather_counts(const PlanArgs &a, int epoch, int *part, int *cnt, 
   __syncthreads();
   int st = 0;
   const unsigned long long t0 = now_ns();
-  for (int64_t c0 = warp; c0 < ntot && st == 0; c0 += (int64_t)kPlanWarps * 32) {
+  // a bad id does not stop the gathering: the generation word may only advance
+  // once every CTA has arrived (and so has read it)
+  for (int64_t c0 = warp; c0 < ntot && !(st & kStTimeout); c0 += (int64_t)kPlanWarps * 32) {
     const int64_t c = c0 + (int64_t)kPlanWarps * lane;  // this lane's chunk in the batch
     bool pend = c < ntot;
     unsigned pending = __ballot_sync(0xffffffffu, pend);
