@@ -1,9 +1,13 @@
 // Data-movement kernels of the MoonEP hot path: zero-copy dispatch, combine,
-// combine-backward and reduce_grad.  All are HBM-bound row moves with O(1)
-// arithmetic per byte; tensor cores are not involved.
+// combine-backward, reduce_grad, and the "next" rows (weight prefetch,
+// dispatch-backward, the copy-through-buffer comparison path).  All are
+// HBM-bound row moves with O(1) arithmetic per byte; tensor cores are not
+// involved.
 //
-// Rows are moved as 16-byte vectors (8 bf16).  One warp owns one token: lane k
-// (< K) holds the token's k-th slot and gate and broadcasts them with shuffles.
+// Rows are moved as 16-byte vectors (8 bf16).  A warp owns a token (dispatch:
+// half a row of one; combine-backward: two warps per token): lane k (< K)
+// holds the token's k-th slot and gate and broadcasts them with shuffles.
+// reduce_grad streams through shared memory with bulk asynchronous copies.
 // Rows whose byte length or base address is not 16-byte aligned take a scalar
 // (one bf16 per lane) path.
 #include <cuda_bf16.h>
