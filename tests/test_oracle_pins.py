@@ -290,6 +290,28 @@ def test_invariants_random(case):
     check_invariants(c, idx, st, t)
 
 
+from hypothesis import given, settings, strategies as hs  # noqa: E402
+
+
+@settings(max_examples=150, deadline=None, derandomize=True)
+@given(R=hs.integers(1, 8), L=hs.integers(1, 4), K=hs.integers(1, 8), S=hs.integers(0, 40),
+       budget_frac=hs.floats(0, 1), mode=hs.integers(0, 1), align=hs.sampled_from([1, 2, 3, 4, 16]),
+       alpha=hs.floats(0, 3), seed=hs.integers(0, 2**31 - 1))
+def test_invariants_property(R, L, K, S, budget_frac, mode, align, alpha, seed):
+    """The contract's invariants over drawn configs: ranks 1-8, 1-4 experts per
+    rank, top-1..8 with ids that may repeat inside a token, budgets 0..L, both
+    modes, alignments 1-16, popularity from uniform to steep Zipf."""
+    E = R * L
+    K = min(K, E)
+    B = int(round(budget_frac * L))
+    p = (np.arange(E) + 1.0) ** -alpha
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(E, size=(R, S, K), p=p / p.sum()).astype(np.int32)
+    c = cfg(R, E, K, S, budget=B, mode=mode, align=align)
+    st, t = oracle.plan(c, idx)
+    check_invariants(c, idx, st, t)
+
+
 def test_invariants_with_repeated_experts_in_a_token():
     idx = uniform_routing(4, 8, 3, 20, seed=5, distinct=False)
     c = cfg(4, 8, 3, 20, budget=1, mode=1, align=2)
