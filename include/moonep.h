@@ -162,9 +162,14 @@ MOONEP_API moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
  *   - Same arguments and results as moonep_plan, without `workspace`.
  *   - Configs whose moonep_workspace_bytes() exceeds the array are rejected
  *     with MOONEP_ERR_UNSUPPORTED before anything is enqueued.
- *   - The first call on a device (with that device current) looks up the
- *     array's device address once; make that first call before any stream
- *     capture.  Nothing is allocated or freed, ever.
+ *   - Host-checkable arguments (config, null or misaligned pointers, size)
+ *     are checked before any CUDA call.
+ *   - The first call in a CUDA context (with the device current) looks up the
+ *     array's device address in that context and caches it under the
+ *     context's id; a device reset or another context on the same device has
+ *     a new id, so the first call there looks it up again.  Make the first
+ *     call in each context before any stream capture.  Nothing is allocated
+ *     or freed, ever.
  *   - All calls on a device share the one array and find it as the previous
  *     call left it; no word of it needs to start at zero (each is written
  *     before it is read in the same call, and the arrival flags carry a

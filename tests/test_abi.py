@@ -79,6 +79,11 @@ def test_null_and_misaligned_pointers_rejected_on_host():
     assert L.moonep_plan(cp, base, base, base, None, 0) == me.ERR_INVALID_ARG
     assert L.moonep_plan(cp, base, base + 16, base, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_plan(cp, base, base, base + 8, base, 0) == me.ERR_INVALID_ARG
+    # the allocation-free plan checks the same arguments before any CUDA call
+    assert L.moonep_plan_static(cp, None, base, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_plan_static(cp, base, None, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_plan_static(cp, base, base, None, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_plan_static(cp, base, base + 16, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_dispatch(cp, base, None, base, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_combine(cp, base, base, None, base, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_combine_backward(cp, base, base, base, base, None, base, base, 0) == \

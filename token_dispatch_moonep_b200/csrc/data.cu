@@ -942,16 +942,7 @@ reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t 
   }
 }
 
-int num_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
-  }
-  return sms;
-}
+int num_sms() { return current_sm_count(); }
 
 unsigned token_grid(int64_t T) {
   int64_t blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;

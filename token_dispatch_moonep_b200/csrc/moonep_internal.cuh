@@ -17,6 +17,18 @@ namespace moonep {
 long long debug_wait_limit_ns();
 int debug_phantom();
 
+// Unique id of the calling thread's current CUDA context (the driver never
+// reuses one within a process, so a device reset or a second context on the
+// same device gives a new id); 0 if it cannot be queried.  Host state that
+// belongs to one context (a kernel's attributes, a device symbol's address)
+// is cached under this id.
+unsigned long long current_context_id();
+
+constexpr int kMaxDevices = 128;  // device ordinals the host-side caches cover
+
+// Streaming multiprocessors of the current device (cached per device; 148 on B200).
+int current_sm_count();
+
 constexpr int kPlanThreads = 512;   // threads per CTA of the plan kernel
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kPairsPerThread = 16;  // most pairs per thread in one plan chunk

@@ -24,6 +24,7 @@
 // so graph replays and reused workspaces need no memset; every wait is bounded
 // in time and reports MOONEP_DEV_TIMEOUT instead of hanging.
 #include <atomic>
+#include <mutex>
 
 #include "moonep_internal.cuh"
 
@@ -1046,6 +1047,52 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
 namespace moonep {
 long long debug_wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 int debug_phantom() { return g_phantom_arrivals.load(std::memory_order_relaxed); }
+
+namespace {
+// driver entry points (no link-time dependency on libcuda)
+typedef int (*CtxGetCurrentFn)(void **ctx);
+typedef int (*CtxGetIdFn)(void *ctx, unsigned long long *id);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fns_once;
+}  // namespace
+
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_fns_once, [] {
+    void *f = nullptr, *g = nullptr;
+    cudaDriverEntryPointQueryResult qf = cudaDriverEntryPointSymbolNotFound, qg = qf;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &qf) == cudaSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &g, cudaEnableDefault, &qg) == cudaSuccess &&
+        qf == cudaDriverEntryPointSuccess && qg == cudaDriverEntryPointSuccess && f && g) {
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(g);
+    }
+    cudaGetLastError();
+  });
+  if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+  void *ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_get_current(&ctx) != 0 || !ctx || g_ctx_get_id(ctx, &id) != 0) return 0;
+  return id;
+}
+
+int current_sm_count() {
+  static std::atomic<int> sms[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return 148;
+  }
+  int v = sms[dev].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return 148;
+    }
+    sms[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
 }  // namespace moonep
 
 extern "C" moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals) {
@@ -1059,12 +1106,41 @@ extern "C" moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phant
 // ------------------------------------------------ allocation-free variant ---
 // Scratch for moonep_plan_static: a fixed device array that lives as long as
 // the library is loaded.  Host code cannot use the symbol itself as a device
-// pointer; its device address is looked up once per device.
+// pointer: its device address is looked up with cudaGetSymbolAddress.  That
+// address belongs to one context's copy of the module (a device reset, or a
+// second context on the same device, loads the module again, possibly
+// elsewhere), so it is cached per device together with the id of the context
+// it was looked up in, and looked up again whenever the current context's id
+// differs.
 static __device__ __align__(256) unsigned char g_plan_scratch[MOONEP_STATIC_WORKSPACE_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 128;
-std::atomic<void *> g_plan_scratch_addr[kMaxDevices];
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void *addr;
+};
+std::mutex g_scratch_mu;
+ScratchAddr g_scratch_addr[kMaxDevices];
+
+// Device address of g_plan_scratch in the current context; nullptr on error.
+void *static_scratch(int dev) {
+  unsigned long long id = current_context_id();
+  {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (id != 0 && g_scratch_addr[dev].ctx_id == id) return g_scratch_addr[dev].addr;
+  }
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  id = current_context_id();  // the lookup makes the device's context current if it was not
+  if (id != 0) {
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    g_scratch_addr[dev] = {id, p};
+  }
+  return p;
+}
 }  // namespace
 
 extern "C" moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const int32_t *topk_idx,
@@ -1072,16 +1148,15 @@ extern "C" moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const 
                                               moonep_stream_t stream) {
   Dims d;
   if (!make_dims(cfg, &d)) return MOONEP_ERR_INVALID_ARG;
+  // every host-checkable argument first: nothing below runs for a bad call
+  if (!plan_arena || !dev_status || (d.N > 0 && !topk_idx) || !aligned256(plan_arena))
+    return MOONEP_ERR_INVALID_ARG;
   if (WsLayout(d).total > (size_t)MOONEP_STATIC_WORKSPACE_BYTES) return MOONEP_ERR_UNSUPPORTED;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOONEP_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOONEP_ERR_UNSUPPORTED;
-  void *scratch = g_plan_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!scratch) {
-    if (cudaGetSymbolAddress(&scratch, g_plan_scratch) != cudaSuccess || !scratch)
-      return MOONEP_ERR_CUDA;
-    g_plan_scratch_addr[dev].store(scratch, std::memory_order_release);
-  }
+  void *scratch = static_scratch(dev);
+  if (!scratch) return MOONEP_ERR_CUDA;
   // the ordinary plan with the static array as its workspace: every scratch
   // word it reads is written earlier in the same call, and its arrival flags
   // are tagged with a per-launch epoch, so nothing needs clearing
