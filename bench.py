@@ -14,7 +14,12 @@ K steps with events only around them (kernels overlap their launch gaps as in
 use); the per-kernel times, the metric and the roofline from a second pass of
 K steps with an event after every kernel.
 Default workload: R=8 ranks, E=256 experts, K=8, S=4096 tokens/rank, H=7168,
-maxvio 0.2, replica budget 32 (training).
+maxvio 0.2, replica budget 32 (training).  The default run then adds, on the
+same line: `sweep` — the forward layer (plan + dispatch + combine) of the same
+shape at maxvio 0.2, 1, 2, 5, 10, 20 over two seeds, with the flatness of the
+layer time; `decode` — the 64-rank inference workload at maxvio 1 and 20; and
+`cpu_baseline` — the CPU oracle on a bounded sample, single-threaded and on
+every host core.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--maxvio M]
     python bench.py --sweep            # maxvio 0.2..20 x 5 seeds, one JSON line per maxvio
@@ -33,6 +38,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -42,10 +48,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from moonep_inputs import (MODE_TRAIN, WORKLOADS, make_dout, make_gates, make_routing,  # noqa: E402
-                           make_x)
+                           make_x, normal_bf16)
 
 METRIC = "dispatch+combine HBM GB/s (% of peak) and plan µs/layer vs maxvio, 1×B200"
 DEFAULT_WORKLOAD = "ep8_e256_k8_s4096_h7168"
+DECODE_WORKLOAD = "ep64_e256_k8_s128_h7168_decode"
+SWEEP_MAXVIO = (0.2, 1.0, 2.0, 5.0, 10.0, 20.0)
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 
@@ -154,6 +162,18 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def merge_clocks(parts):
+    """One clocks record over several sampled regions (median of the medians, all reasons)."""
+    parts = [c for c in parts if c]
+    if not parts:
+        return None
+    return {"sm_mhz": statistics.median(c["sm_mhz"] for c in parts),
+            "sm_min_mhz": min(c["sm_mhz"] for c in parts),
+            "sm_max_mhz": max(c["sm_max_mhz"] for c in parts),
+            "samples": sum(c["samples"] for c in parts),
+            "reasons": sorted(set().union(*[set(c["reasons"]) for c in parts]))}
+
+
 # ------------------------------------------------------------- GPU layer ---
 class Layer:
     """Device buffers and the per-step call sequence of one MoE layer."""
@@ -168,12 +188,8 @@ class Layer:
         self.cfg = me.Config.of(w)
         self.NvS = me.moonep_nvs(self.cfg)
         T = R * S
-        idx, self.alpha, self.maxvio = make_routing(R, E, K, S, maxvio, seed)
-        gates = make_gates(R, S, K, seed)
-        # pinned host copies (for the end-to-end measurement) and device copies
         pin = torch.cuda.is_available()
-        self.h_idx = torch.from_numpy(idx.ravel().copy())
-        self.h_gates = torch.from_numpy(gates.ravel().copy())
+        self.pin = pin
         if host_inputs:
             self.h_x = torch.from_numpy(make_x(R, S, H, seed).reshape(-1).view(np.int16))
             self.h_dout = (torch.from_numpy(make_dout(R, S, H, seed).reshape(-1).view(np.int16))
@@ -184,13 +200,12 @@ class Layer:
             self.h_dout = (torch.randn(T * H, generator=g, device=device).to(torch.bfloat16)
                            .view(torch.int16).cpu() if self.train else None)
         if pin:
-            self.h_idx = self.h_idx.pin_memory()
-            self.h_gates = self.h_gates.pin_memory()
             self.h_x = self.h_x.pin_memory()
             if self.h_dout is not None:
                 self.h_dout = self.h_dout.pin_memory()
-        self.idx = self.h_idx.to(device)
-        self.gates = self.h_gates.to(device)
+        self.idx = torch.empty(T * K, dtype=torch.int32, device=device)
+        self.gates = torch.empty(T * K, dtype=torch.float32, device=device)
+        self.set_routing(maxvio, seed)
         self.x = self.h_x.to(device)
         self.recv = torch.empty(R * self.NvS * H, dtype=torch.int16, device=device)
         self.out = torch.empty(T * H, dtype=torch.int16, device=device)
@@ -217,9 +232,22 @@ class Layer:
         else:
             self.P = 0
             self.h_out = torch.empty(T * H, dtype=torch.int16).pin_memory() if pin else None
-        self.launches_per_step = 3 + (4 if self.train else 0)  # the plan is one kernel
-        self.n_local = self.n_rep_exp = 0
+        self.n_local = self.n_rep_exp = self.n_piece = self.n_remote = 0
         self.e2e_bufs = None
+
+    def set_routing(self, maxvio, seed):
+        """New router output (tuned to `maxvio`) and gates in the same device buffers."""
+        torch, w = self.torch, self.w
+        idx, self.alpha, self.maxvio = make_routing(w.R, w.E, w.K, w.S, maxvio, seed)
+        gates = make_gates(w.R, w.S, w.K, seed)
+        self.h_idx = torch.from_numpy(idx.ravel().copy())
+        self.h_gates = torch.from_numpy(gates.ravel().copy())
+        if self.pin:
+            self.h_idx = self.h_idx.pin_memory()
+            self.h_gates = self.h_gates.pin_memory()
+        self.idx.copy_(self.h_idx)
+        self.gates.copy_(self.h_gates)
+        self.torch.cuda.synchronize()
 
     def alloc_e2e(self):
         """Second set of input and output buffers so copies of one step overlap another."""
@@ -238,19 +266,21 @@ class Layer:
             self.e2e_bufs = ([first, second], h_out, h_dg)
         return self.e2e_bufs
 
-    def ops(self, buf=None):
-        """The step's ABI calls; `buf` selects an input/output buffer set (default: the first)."""
+    def ops(self, buf=None, forward_only=False):
+        """The step's ABI calls; `buf` selects an input/output buffer set (default: the
+        first); `forward_only` keeps plan, dispatch and combine."""
         me, c = self.me, self.cfg
+        train = self.train and not forward_only
         b = buf or dict(idx=self.idx, gates=self.gates, x=self.x, out=self.out,
                         dout=getattr(self, "dout", None), dg=getattr(self, "dg", None))
         seq = [("plan", lambda: me.moonep_plan(c, b["idx"], self.arena, self.ws, self.status))]
-        if self.train:
+        if train:
             seq += [("prefetch", lambda: me.moonep_prefetch_weight(c, self.arena, self.weights, self.rep_w,
                                                                    self.P, self.status))]
         seq += [("dispatch", lambda: me.moonep_dispatch(c, self.arena, b["x"], self.recv, self.status)),
                ("combine", lambda: me.moonep_combine(c, self.arena, self.recv, b["gates"], b["out"],
                                                      self.status))]
-        if self.train:
+        if train:
             seq += [("combine_bwd", lambda: me.moonep_combine_backward(
                         c, self.arena, b["dout"], self.recv, b["gates"], self.dy, b["dg"],
                         self.status)),
@@ -266,16 +296,16 @@ class Layer:
         self.n_local, self.n_rep_exp = int(sc[2]), int(sc[3])
         self.n_piece, self.n_remote = int(sc[0]), int(sc[1])
 
-    def bytes(self):
+    def bytes(self, forward_only=False):
         w = self.w
         b = algorithmic_bytes(w.R, w.S, w.K, w.H, self.n_local, self.n_rep_exp, self.P)
-        if not self.train:
+        if not self.train or forward_only:
             for k in ("combine_bwd", "reduce_grad", "prefetch", "dispatch_bwd"):
                 b.pop(k)
         return b
 
 
-def time_steps(layer, steps, warmup, barrier=None):
+def time_steps(layer, steps, warmup, barrier=None, ops=None):
     """Warm up, then time `steps` steps twice on the current stream.
 
     Pass 1 is the timed region of the result line: events only before the first
@@ -285,7 +315,8 @@ def time_steps(layer, steps, warmup, barrier=None):
     the per-kernel breakdown; an event between two kernels ends that overlap,
     so per-kernel times carry a few microseconds more than pass 1 accounts for."""
     torch = layer.torch
-    ops = layer.ops()
+    ops = ops or layer.ops()
+    layer.status.zero_()
     for _ in range(warmup):
         for _, fn in ops:
             fn()
@@ -400,50 +431,252 @@ def whole_job_gbs(bytes_per_rank, world, ms):
     return bytes_per_rank * world / (ms * 1e-3) / 1e9
 
 
+def workload_config(w, maxvio, alpha, world, scaled=False):
+    """The `config` object of the result line (shared by both arms)."""
+    NvS = w.S * w.K + (w.align - 1) * min(w.E, w.S * w.K)
+    train = w.mode == MODE_TRAIN
+    return {"workload": w.name + (f"/S{w.S}" if scaled else ""),
+            "R": w.R, "E": w.E, "K": w.K, "S": w.S, "H": w.H, "budget": w.budget,
+            "mode": "train" if train else "infer",
+            "maxvio": round(maxvio, 4), "zipf_alpha": round(alpha, 4),
+            "step": ("plan+prefetch+dispatch+combine+combine_bwd+dispatch_bwd+reduce_grad"
+                     if train else "plan+dispatch+combine"),
+            "grad_elems_per_expert": (w.P or 2048 * w.H) if train else 0,
+            "l2": "inputs larger than L2 (x %.0f MB, dispatch buffer %.0f MB); no flush"
+                  % (w.R * w.S * w.H * 2 / 1e6, w.R * NvS * w.H * 2 / 1e6),
+            "parallelism": f"{world} independent replica(s), one per GPU"}
+
+
+# ------------------------------------------------------ sweep and decode ---
+def forward_pass(layer, steps, warmup):
+    """Plan + dispatch + combine of the layer's current routing: per-kernel medians and
+    the overlapped layer time (pass 1 of time_steps)."""
+    ops = layer.ops(forward_only=True)
+    total_ms, per, clocks, st = time_steps(layer, steps, warmup, ops=ops)
+    b = layer.bytes(forward_only=True)
+    med = {k: statistics.median(v) for k, v in per.items()}
+    return {"maxvio": round(layer.maxvio, 4), "alpha": round(layer.alpha, 4),
+            "plan_us": med["plan"] * 1e3,
+            "dispatch_GBs": b["dispatch"] / med["dispatch"] / 1e6,
+            "combine_GBs": b["combine"] / med["combine"] / 1e6,
+            "layer_us": 1e3 * total_ms / steps,
+            "layer_us_kernel_events": 1e3 * (med["plan"] + med["dispatch"] + med["combine"]),
+            "pieces": layer.n_piece, "remote": layer.n_remote, "status": st}, clocks
+
+
+def compact_sweep(layer, seeds, steps, warmup, targets=SWEEP_MAXVIO):
+    """The forward layer of `layer`'s shape across router imbalance, reusing its buffers."""
+    peak, _ = hbm_peak()
+    rows, clocks = [], []
+    for mv in targets:
+        per_seed = []
+        for seed in seeds:
+            layer.set_routing(mv, seed)
+            r, c = forward_pass(layer, steps, warmup)
+            r["seed"] = seed
+            per_seed.append(r)
+            clocks.append(c)
+        row = {"target_maxvio": mv}
+        for k in ("maxvio", "plan_us", "dispatch_GBs", "combine_GBs", "layer_us",
+                  "layer_us_kernel_events", "pieces"):
+            row[k] = statistics.mean(r[k] for r in per_seed)
+        row["status"] = max(r["status"] for r in per_seed)
+        row["seeds"] = per_seed
+        rows.append(row)
+    lay = [r["layer_us"] for r in rows]
+    plan = [r["plan_us"] for r in rows]
+    return {"workload": layer.w.name, "seeds": list(seeds), "steps": steps,
+            "layer": "plan+dispatch+combine, overlapped launches (events only around the steps)",
+            "flatness": max(lay) / min(lay), "plan_flatness": max(plan) / min(plan),
+            "peak_GBs": peak, "rows": rows, "clocks": merge_clocks(clocks)}
+
+
+def decode_runs(device, steps, warmup, maxvios=(1.0, 20.0), seed=0):
+    """The 64-rank inference workload: plan + dispatch + combine µs per maxvio."""
+    w = WORKLOADS[DECODE_WORKLOAD]
+    layer = Layer(w, maxvios[0], seed, device, with_backward=False, host_inputs=False)
+    out, clocks = [], []
+    for mv in maxvios:
+        layer.set_routing(mv, seed)
+        r, c = forward_pass(layer, steps, warmup)
+        out.append(r)
+        clocks.append(c)
+    b = layer.bytes(forward_only=True)
+    res = {"workload": w.name, "seed": seed, "steps": steps,
+           "bytes_dispatch_combine": b["dispatch"] + b["combine"],
+           "rows": out, "clocks": merge_clocks(clocks)}
+    del layer
+    return res
+
+
 # ------------------------------------------------------------ CPU oracle ---
-def oracle_sample_run(w, maxvio, seed, s_sample, budget_s=10.0, min_reps=1):
-    """Time the CPU oracle (plan + dispatch + combine) on the first `s_sample` tokens of
-    every rank of the workload's routing, repeated until `budget_s` seconds pass."""
-    import oracle
-    R, E, K, H = w.R, w.E, w.K, w.H
-    idx, _, _ = make_routing(R, E, K, w.S, maxvio, seed)
-    idx = np.ascontiguousarray(idx[:, :s_sample, :])
-    gates = np.ascontiguousarray(make_gates(R, w.S, K, seed)[:, :s_sample, :])
-    x = make_x(R, s_sample, H, seed).reshape(R * s_sample, H)
-    cfg = oracle.Config(R=R, E=E, K=K, S=s_sample, H=H, budget=w.budget, mode=w.mode)
-    b = algorithmic_bytes(R, s_sample, K, H)
-    reps, t_plan, t_dc = 0, 0.0, 0.0
-    t_start = time.perf_counter()
-    while reps < min_reps or time.perf_counter() - t_start < budget_s:
-        a = time.perf_counter()
-        st, t = oracle.plan(cfg, idx)
-        m = time.perf_counter()
-        recv = oracle.dispatch(cfg, t["slot_of"], x)
-        oracle.combine(cfg, t["slot_of"], recv, gates)
-        e = time.perf_counter()
-        t_plan += m - a
-        t_dc += e - m
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _run_threads(fn, parts):
+    """fn(part) on one thread per part (the oracle's C calls release the GIL)."""
+    if len(parts) == 1:
+        fn(parts[0])
+        return
+    ths = [threading.Thread(target=fn, args=(p,)) for p in parts]
+    for t in ths:
+        t.start()
+    for t in ths:
+        t.join()
+
+
+def _time_until(fn, min_s):
+    """Repeat fn until at least min_s seconds have passed; (reps, seconds)."""
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        fn()
         reps += 1
-    gbs = (b["dispatch"] + b["combine"]) * reps / t_dc / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "plan_us": t_plan / reps * 1e6, "reps": reps, "seconds": t_dc + t_plan,
-            "sample": f"first {s_sample} of {w.S} tokens on each of the {R} ranks of the "
-                      f"same seeded routing (maxvio {maxvio}), planned as one layer; "
-                      f"plan + dispatch + combine, single-threaded C, repeated {reps}x"}
+        el = time.perf_counter() - t0
+        if el >= min_s:
+            return reps, el
+
+
+class OracleSample:
+    """The unchanged CPU oracle on a bounded sample of a workload: the first `s` tokens of
+    every rank of the same seeded routing, planned as one layer of S = s tokens, and
+    expert-gradient / weight rows cut to their first `p` elements."""
+
+    def __init__(self, w, maxvio, seed, s, p=1 << 18):
+        import oracle
+        self.o = oracle
+        R, E, K, H, B = w.R, w.E, w.K, w.H, w.budget
+        idx, _, _ = make_routing(R, E, K, w.S, maxvio, seed)
+        self.idx = np.ascontiguousarray(idx[:, :s, :])
+        self.gates = np.ascontiguousarray(make_gates(R, w.S, K, seed)[:, :s, :]).reshape(R * s, K)
+        self.x = make_x(R, s, H, seed).reshape(R * s, H)
+        self.dout = make_dout(R, s, H, seed).reshape(R * s, H)
+        self.cfg = oracle.Config(R=R, E=E, K=K, S=s, H=H, budget=w.budget, mode=w.mode)
+        self.R, self.E, self.K, self.H, self.B, self.s, self.P = R, E, K, H, B, s, p
+        self.train = w.mode == MODE_TRAIN
+        st, self.t = oracle.plan(self.cfg, self.idx)
+        self.slot_of = self.t["slot_of"]
+        self.NvS = int(self.t["nvs"][0])
+        self.recv = np.zeros((R * self.NvS, H), np.uint16)
+        self.out = np.zeros((R * s, H), np.uint16)
+        self.dy = np.zeros((R * self.NvS, H), np.uint16)
+        local = self.t["piece_wslot"] >= 0
+        self.n_local = int(local.sum())
+        self.rep_experts = np.unique(self.t["piece_expert"][local])
+        if self.train:
+            # N(0,1) rows (no subnormal values, which would slow the host arithmetic down);
+            # only the slots of local pieces are ever read
+            self.home = normal_bf16((E, p), seed, stream=21)
+            self.rep = np.zeros((R, max(B, 1), p), np.uint16)
+            li = np.nonzero(local)[0]
+            rows = normal_bf16((max(len(li), 1), p), seed, stream=22)
+            for j, i in enumerate(li):
+                self.rep[self.t["piece_rank"][i], self.t["piece_wslot"][i]] = rows[j]
+            self.weights = self.home.copy()
+            self.rep_w = np.zeros_like(self.rep)
+
+    def bytes(self):
+        return algorithmic_bytes(self.R, self.s, self.K, self.H, self.n_local,
+                                 len(self.rep_experts), self.P)
+
+    def kernels(self):
+        """name -> callable(n_threads) running that step of the oracle once."""
+        o, c, K, H = self.o, self.cfg, self.K, self.H
+        T = self.R * self.s
+
+        def token_parts(n):
+            return [p for p in np.array_split(np.arange(T, dtype=np.int64), n) if p.size]
+
+        def dispatch(n):
+            def part(tk):
+                t0, t1 = int(tk[0]), int(tk[-1]) + 1
+                sub = o.Config(R=1, E=c.E, K=K, S=t1 - t0, H=H, budget=c.budget, mode=c.mode)
+                o.dispatch(sub, self.slot_of[t0 * K:t1 * K], self.x[t0:t1], self.recv)
+            _run_threads(part, token_parts(n))
+
+        def combine(n):
+            _run_threads(lambda tk: o.combine(c, self.slot_of, self.recv, self.gates, tk),
+                         token_parts(n))
+
+        def combine_bwd(n):
+            _run_threads(lambda tk: o.combine_backward(c, self.slot_of, self.dout, self.recv,
+                                                       self.gates, tk), token_parts(n))
+
+        def dispatch_bwd(n):
+            _run_threads(lambda tk: o.dispatch_backward(c, self.slot_of, self.dy, tk),
+                         token_parts(n))
+
+        def expert_parts(n):
+            groups = [g for g in np.array_split(self.rep_experts, n) if g.size]
+            out = []
+            for g in groups:
+                m = np.isin(self.t["piece_expert"], g)
+                out.append({k: self.t[k][m] for k in ("piece_expert", "piece_rank", "piece_wslot")})
+            return out or [{k: self.t[k][:0] for k in ("piece_expert", "piece_rank",
+                                                        "piece_wslot")}]
+
+        def reduce_grad(n):
+            _run_threads(lambda tb: o.reduce_grad(c, tb, self.rep, self.home, inplace=True),
+                         expert_parts(n))
+
+        def prefetch(n):
+            _run_threads(lambda tb: o.prefetch_weight(c, tb, self.weights, self.rep_w, inplace=True),
+                         expert_parts(n))
+
+        ks = {"dispatch": dispatch, "combine": combine}
+        if self.train:
+            ks.update(prefetch=prefetch, combine_bwd=combine_bwd, dispatch_bwd=dispatch_bwd,
+                      reduce_grad=reduce_grad)
+        return ks
+
+
+def oracle_baseline(w, maxvio, seed, s_sample, min_s=1.0):
+    """The CPU oracle, as it stands, on a bounded sample: the plan single-threaded (its
+    algorithm is sequential) and every data step single-threaded and on every host core
+    (threads over disjoint tokens or experts).  GB/s of the same algorithmic bytes."""
+    smp = OracleSample(w, maxvio, seed, s_sample)
+    cores = host_cores()
+    b = smp.bytes()
+    t0 = time.perf_counter()
+    reps, el = _time_until(lambda: smp.o.plan(smp.cfg, smp.idx), min_s / 2)
+    plan_us = el / reps * 1e6
+    single, multi = {}, {}
+    for name, fn in smp.kernels().items():
+        r1, e1 = _time_until(lambda: fn(1), min_s)
+        single[name] = b[name] * r1 / e1 / 1e9
+        rn, en = _time_until(lambda: fn(cores), min_s)
+        multi[name] = b[name] * rn / en / 1e9
+    dc = b["dispatch"] + b["combine"]
+    value = dc / (b["dispatch"] / multi["dispatch"] + b["combine"] / multi["combine"])
+    value_1 = dc / (b["dispatch"] / single["dispatch"] + b["combine"] / single["combine"])
+    return {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "single_thread_value": value_1, "plan_us_single_thread": plan_us,
+            "single_thread": single, "all_cores": multi,
+            "seconds": time.perf_counter() - t0,
+            "sample": f"first {s_sample} of {w.S} tokens on each of the {w.R} ranks of the same "
+                      f"seeded routing (maxvio {maxvio}), planned as one layer of S={s_sample}; "
+                      f"expert gradient / weight rows cut to {smp.P} elements; every step of "
+                      f"the layer timed single-threaded and on {cores} threads (disjoint tokens "
+                      f"or experts), each repeated for >= {min_s:.1f} s; value = dispatch + "
+                      f"combine on all {cores} threads"}
 
 
 def run_reference(args, rank, world):
-    """The reference arm: the CPU oracle, on the same metric, on a bounded sample per step."""
+    """The reference arm: the CPU oracle on every host core, same metric and config, on a
+    bounded sample of the workload per step."""
     if rank != 0:
         return 0
     w = WORKLOADS[args.workload]
     mv = args.maxvio if args.maxvio is not None else w.maxvio[0]
-    s_sample = max(1, min(w.S, 8 if w.H >= 4096 else 64))
+    s_sample = max(1, min(w.S, 64 if w.H >= 4096 else 256))
     import oracle
     R, E, K, H = w.R, w.E, w.K, w.H
-    idx, _, _ = make_routing(R, E, K, w.S, mv, args.seed)
+    cores = host_cores()
+    idx, alpha, realized = make_routing(R, E, K, w.S, mv, args.seed)
     gates = make_gates(R, w.S, K, args.seed)
-    x_full = None
     b = algorithmic_bytes(R, s_sample, K, H)
     cfg = oracle.Config(R=R, E=E, K=K, S=s_sample, H=H, budget=w.budget, mode=w.mode)
     times, plan_t = [], []
@@ -453,13 +686,22 @@ def run_reference(args, rank, world):
         # step s uses the s-th slice of s_sample tokens of every rank (wrapping)
         lo = (step * s_sample) % max(1, w.S - s_sample + 1)
         si = np.ascontiguousarray(idx[:, lo:lo + s_sample, :])
-        sg = np.ascontiguousarray(gates[:, lo:lo + s_sample, :])
+        sg = np.ascontiguousarray(gates[:, lo:lo + s_sample, :]).reshape(R * s_sample, K)
         x = make_x(R, s_sample, H, args.seed + step).reshape(R * s_sample, H)
         a = time.perf_counter()
         st, t = oracle.plan(cfg, si)
         m = time.perf_counter()
-        recv = oracle.dispatch(cfg, t["slot_of"], x)
-        oracle.combine(cfg, t["slot_of"], recv, sg)
+        slot_of = t["slot_of"]
+        recv = np.zeros((R * int(t["nvs"][0]), H), np.uint16)
+        parts = [p for p in np.array_split(np.arange(R * s_sample, dtype=np.int64), cores) if p.size]
+
+        def disp(tk):
+            t0, t1 = int(tk[0]), int(tk[-1]) + 1
+            sub = oracle.Config(R=1, E=E, K=K, S=t1 - t0, H=H, budget=w.budget, mode=w.mode)
+            oracle.dispatch(sub, slot_of[t0 * K:t1 * K], x[t0:t1], recv)
+
+        _run_threads(disp, parts)
+        _run_threads(lambda tk: oracle.combine(cfg, slot_of, recv, sg, tk), parts)
         e = time.perf_counter()
         if step >= args.warmup:
             times.append(e - m)
@@ -469,17 +711,16 @@ def run_reference(args, rank, world):
             break
     gbs = (b["dispatch"] + b["combine"]) * done / sum(times) / 1e9
     sample = (f"per step {s_sample} tokens on each of the {R} ranks (a slice of the seeded "
-              f"{args.workload} routing, maxvio {mv}), planned as one layer; plan + dispatch + "
-              "combine in the single-threaded C oracle")
+              f"{args.workload} routing, maxvio {mv}), planned as one layer (single-threaded); "
+              f"dispatch + combine in the C oracle on {cores} threads over disjoint tokens")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
         "steps": done, "warmup": args.warmup, "ms_per_step": 1e3 * (sum(times) + sum(plan_t)) / done,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": {"workload": args.workload, "maxvio": mv,
-                                        "sample_tokens_per_rank": s_sample},
+        "data": "synthetic", "config": workload_config(w, realized, alpha, world),
         "plan_us_per_layer": 1e6 * sum(plan_t) / done,
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample, "sample_tokens_per_rank": s_sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -503,6 +744,10 @@ def main():
     ap.add_argument("--scale-s", type=int, default=1, help="divide S (tokens/rank) by this (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="headline line only: no compact sweep, no decode workload")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="timed steps per point of the compact sweep and the decode runs")
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     args = ap.parse_args()
 
@@ -561,6 +806,10 @@ def main():
     roof = {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["GBs"], "peak": peak,
             "unit": "GB/s", "frac": kern[dom]["GBs"] / peak, "traffic": traffic,
             "peak_source": f"{peak_src} copy bandwidth"}
+    launches = len(layer.ops()) * args.steps
+    headline_cfg = workload_config(w, layer.maxvio, layer.alpha, world, scaled=args.scale_s > 1)
+    replicas = {"pieces": layer.n_piece, "local": layer.n_local, "remote": layer.n_remote,
+                "experts_replicated": layer.n_rep_exp}
 
     e2e = None
     if not args.no_e2e:
@@ -573,9 +822,18 @@ def main():
                "how": "inputs copied in and results read back every step, overlapped with "
                       "the previous/next step's compute (two buffer sets)"}
 
+    sweep = decode = None
+    if not args.no_extra and args.scale_s <= 1 and world == 1 and w.name == DEFAULT_WORKLOAD:
+        ex_warm = max(3, min(args.warmup, 5))
+        sweep = compact_sweep(layer, (0, 1), args.extra_steps, ex_warm)
+        del layer
+        torch.cuda.empty_cache()
+        decode = decode_runs(device, args.extra_steps, ex_warm)
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = oracle_sample_run(w, mv, args.seed, s_sample=min(w.S, 64 if w.H >= 4096 else 256))
+        cpu = oracle_baseline(w, mv, args.seed, s_sample=min(w.S, 128 if w.H >= 4096 else 256))
 
     if rank == 0:
         line = {
@@ -583,28 +841,20 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": w.name + (f"/S{w.S}" if args.scale_s > 1 else ""),
-                       "R": w.R, "E": w.E, "K": w.K, "S": w.S, "H": w.H, "budget": w.budget,
-                       "mode": "train" if w.mode == MODE_TRAIN else "infer",
-                       "maxvio": round(layer.maxvio, 4), "zipf_alpha": round(layer.alpha, 4),
-                       "step": ("plan+prefetch+dispatch+combine+combine_bwd+dispatch_bwd+reduce_grad"
-                                if layer.train else "plan+dispatch+combine"),
-                       "grad_elems_per_expert": layer.P,
-                       "l2": "inputs larger than L2 (x %.0f MB, dispatch buffer %.0f MB); no flush"
-                             % (layer.x.numel() * 2 / 1e6, layer.recv.numel() * 2 / 1e6),
-                       "parallelism": f"{world} independent replica(s), one per GPU"},
+            "config": headline_cfg,
             "pct_of_peak": {"measured": value / peak, "nominal_8TBs": value / NOMINAL_HBM_GBS},
             "plan_us_per_layer": kern["plan"]["ms"] * 1e3,
             "layer_us": 1e3 * (kern["plan"]["ms"] + kern["dispatch"]["ms"] + kern["combine"]["ms"]),
             "kernels": kern,
-            "replicas": {"pieces": layer.n_piece, "local": layer.n_local, "remote": layer.n_remote,
-                         "experts_replicated": layer.n_rep_exp},
+            "replicas": replicas,
             "device_status": st,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": layer.launches_per_step * args.steps,
+            "gpu_launches": launches,
             "clocks": clocks,
+            "sweep": sweep,
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -665,40 +915,12 @@ def run_compare_copy(args, w, device):
 def run_sweep(args, w, device):
     """Plan µs and dispatch/combine GB/s per maxvio (5 seeds each), plus flatness.
     Forward only (plan + dispatch + combine), the per-layer time the pages plot."""
-    rows = []
-    peak, _ = hbm_peak()
-    targets = (0.2, 1.0, 2.0, 5.0, 10.0, 20.0) if args.maxvio is None else (args.maxvio,)
-    seeds = (0, 1, 2, 3, 4)
-    for mv in targets:
-        per_seed = []
-        for seed in seeds:
-            layer = Layer(w, mv, seed, device, with_backward=False, host_inputs=False)
-            total_ms, per, clocks, st = time_steps(layer, max(20, args.steps // 10), args.warmup)
-            b = layer.bytes()
-            med = {k: statistics.median(v) for k, v in per.items()}
-            per_seed.append({"seed": seed, "maxvio": layer.maxvio, "alpha": layer.alpha,
-                             "plan_us": med["plan"] * 1e3,
-                             "dispatch_GBs": b["dispatch"] / med["dispatch"] / 1e6,
-                             "combine_GBs": b["combine"] / med["combine"] / 1e6,
-                             "layer_us": 1e3 * (med["plan"] + med["dispatch"] + med["combine"]),
-                             "pieces": layer.n_piece, "status": st, "clocks": clocks})
-            del layer
-            import torch
-            torch.cuda.empty_cache()
-        row = {"target_maxvio": mv,
-               "maxvio": statistics.mean(r["maxvio"] for r in per_seed),
-               "plan_us": statistics.mean(r["plan_us"] for r in per_seed),
-               "dispatch_GBs": statistics.mean(r["dispatch_GBs"] for r in per_seed),
-               "combine_GBs": statistics.mean(r["combine_GBs"] for r in per_seed),
-               "layer_us": statistics.mean(r["layer_us"] for r in per_seed),
-               "pieces": statistics.mean(r["pieces"] for r in per_seed),
-               "seeds": per_seed}
-        rows.append(row)
+    layer = Layer(w, SWEEP_MAXVIO[0], 0, device, with_backward=False, host_inputs=False)
+    targets = SWEEP_MAXVIO if args.maxvio is None else (args.maxvio,)
+    res = compact_sweep(layer, (0, 1, 2, 3, 4), max(20, args.steps // 10), args.warmup, targets)
+    for row in res["rows"]:
         print(json.dumps({k: v for k, v in row.items() if k != "seeds"}), flush=True)
-    lay = [r["layer_us"] for r in rows]
-    print(json.dumps({"sweep": w.name, "flatness_max_over_min_layer_us": max(lay) / min(lay),
-                      "layer_us": lay, "peak_GBs": peak,
-                      "rows": rows}), flush=True)
+    print(json.dumps(res), flush=True)
     return 0
 
 

@@ -196,10 +196,14 @@ def combine_backward(cfg: Config, slot_of: np.ndarray, dout: np.ndarray, y: np.n
     return dy, dg
 
 
-def reduce_grad(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray, home: np.ndarray
-                ) -> np.ndarray:
-    """New home gradients (bf16 bits [E, P]); ``rep`` is [R, budget, P]."""
-    home = np.array(home, dtype=np.uint16, copy=True, order="C")
+def reduce_grad(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray, home: np.ndarray,
+                inplace: bool = False) -> np.ndarray:
+    """New home gradients (bf16 bits [E, P]); ``rep`` is [R, budget, P].  With
+    ``inplace`` the result is written into ``home`` itself (a C-contiguous uint16
+    array) instead of a copy."""
+    if not (inplace and isinstance(home, np.ndarray) and home.dtype == np.uint16
+            and home.flags["C_CONTIGUOUS"] and home.flags["WRITEABLE"]):
+        home = np.array(home, dtype=np.uint16, copy=True, order="C")
     rep = _c(rep, np.uint16)
     P = home.shape[-1]
     pe = _c(tables["piece_expert"], np.int32)
@@ -222,9 +226,12 @@ def dispatch_backward(cfg: Config, slot_of: np.ndarray, drecv: np.ndarray,
 
 
 def prefetch_weight(cfg: Config, tables: Dict[str, np.ndarray], w: np.ndarray,
-                    rep_w: np.ndarray) -> np.ndarray:
-    """Replica weight slots after the prefetch (bf16 bits [R, budget, W]); ``w`` is [E, W]."""
-    rep_w = np.array(rep_w, dtype=np.uint16, copy=True, order="C")
+                    rep_w: np.ndarray, inplace: bool = False) -> np.ndarray:
+    """Replica weight slots after the prefetch (bf16 bits [R, budget, W]); ``w`` is [E, W].
+    With ``inplace`` the slots are written into ``rep_w`` itself (C-contiguous uint16)."""
+    if not (inplace and isinstance(rep_w, np.ndarray) and rep_w.dtype == np.uint16
+            and rep_w.flags["C_CONTIGUOUS"] and rep_w.flags["WRITEABLE"]):
+        rep_w = np.array(rep_w, dtype=np.uint16, copy=True, order="C")
     ww = _c(w, np.uint16)
     pe = _c(tables["piece_expert"], np.int32)
     pr = _c(tables["piece_rank"], np.int32)

@@ -76,3 +76,46 @@ def test_reference_arm_runs_on_rank_zero_only(rank):
         assert d["e2e"]["h2d_bytes_per_step"] == 0
     else:
         assert lines == []
+
+
+def test_oracle_baseline_threads_cover_the_same_work():
+    """The threaded CPU baseline splits each step over disjoint tokens or experts: every
+    thread count must leave exactly the single-threaded results behind."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    from moonep_inputs import WORKLOADS
+    w = WORKLOADS["ep8_e32_k4_s256_h512"]
+    res = {}
+    for n in (1, 3, 8):
+        smp = bench.OracleSample(w, 5.0, 0, s=40, p=4096)
+        assert smp.n_local > 0
+        ks = smp.kernels()
+        for name in ("dispatch", "reduce_grad", "prefetch"):
+            ks[name](n)
+        res[n] = (smp.recv.copy(), smp.home.copy(), smp.rep_w.copy())
+    for n in (3, 8):
+        for a, b in zip(res[1], res[n]):
+            assert np.array_equal(a, b)
+    smp = bench.OracleSample(w, 5.0, 0, s=40, p=4096)
+    ks = smp.kernels()
+    for name in ("combine", "combine_bwd", "dispatch_bwd"):
+        ks[name](4)  # runs over every token without error
+
+
+def test_reference_line_carries_the_gpu_arm_config():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "ep8_e32_k4_s256_h512", "--steps", "2", "--warmup", "1",
+                        "--reference-budget-s", "5"], capture_output=True, text=True, env=env,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    sys.path.insert(0, ROOT)
+    import bench
+    from moonep_inputs import WORKLOADS, make_routing
+    w = WORKLOADS["ep8_e32_k4_s256_h512"]
+    _, alpha, mv = make_routing(w.R, w.E, w.K, w.S, w.maxvio[0], 0)
+    assert d["config"] == bench.workload_config(w, mv, alpha, 1)
+    assert d["cpu_baseline"]["cores"] == bench.host_cores()

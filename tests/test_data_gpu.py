@@ -2,8 +2,12 @@
 
 Bar: dispatched rows bit-exact (and padding rows untouched); combine,
 combine-backward and reduce_grad within 1e-3 norm-relative error
-(max |gpu - ref| / max |ref|) with fp32 accumulation.  The bit-identical
-fraction is also asserted where both sides round the same fp32 value.
+(max |gpu - ref| / max |ref|) with fp32 accumulation.  Where both sides round
+the same fp32 value, computed with the same operations in the same order
+(combine: fused multiply-adds in ascending k; dY: one product;
+dispatch-backward: additions in ascending k; reduce_grad: additions in piece
+order), the results must also be bit-identical.  dgate (an fp32 dot product
+on the GPU, fp64 in the oracle) is held to 1e-3 only.
 """
 import numpy as np
 import pytest
@@ -15,6 +19,12 @@ from tests.gpu_util import POISON, configs, gpu_plan, rel_err, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-3
+
+
+def _exact(got, ref):
+    """The contract's 1e-3 norm-relative bar, and bit-identity (same fp32 steps)."""
+    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    assert np.array_equal(got, ref), int((got != ref).sum())
 
 
 def _setup(R, E, K, S, H, mv=3.0, seed=0, budget=None, mode=0, align=1):
@@ -113,8 +123,7 @@ def test_combine_matches_oracle(shape):
     if ref.size == 0:
         assert got.size == 0
         return
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
 
 
 @pytest.mark.parametrize("shape", SHAPES[:3])
@@ -128,7 +137,7 @@ def test_round_trip_identity_expert(shape):
     w = make_gates(R, S, K, seed=4)
     got = _combine(cfg, arena, recv, w)
     ref = oracle.combine(ocfg, ot["slot_of"], oracle.dispatch(ocfg, ot["slot_of"], x), w)
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
+    _exact(got, ref)
     exact = w.reshape(R * S, K).astype(np.float64).sum(1, keepdims=True) * bf16_bits_to_f32(x)
     assert rel_err(bf16_bits_to_f32(got), exact) <= 2 ** -7
 
@@ -163,8 +172,7 @@ def test_combine_backward_matches_oracle(shape):
         return
     so = ot["slot_of"]
     got_rows = dy[so].reshape(R * S, K, H)
-    assert rel_err(bf16_bits_to_f32(got_rows), bf16_bits_to_f32(ref_dy)) <= TOL
-    assert (got_rows == ref_dy).mean() >= 0.999
+    _exact(got_rows, ref_dy)
     assert (dy[ot["slot_src"] < 0] == POISON).all()
     assert rel_err(dg.reshape(R * S, K), ref_dg) <= TOL
 
@@ -191,8 +199,7 @@ def test_reduce_grad_matches_oracle(shape):
     home = normal_bf16((E, P), seed=6, stream=12)
     got = _reduce(cfg, arena, rep, home, P)
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
 
 
 def test_reduce_grad_gradient_equivalence_exact():
@@ -241,8 +248,7 @@ def test_reduce_grad_expert_with_many_pieces():
     home = normal_bf16((E, P), seed=7, stream=12)
     got = _reduce(cfg, arena, rep, home, P)
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
 
 
 @pytest.mark.parametrize("R,P", [(80, 10000), (80, 8), (80, 13)])
@@ -263,8 +269,7 @@ def test_reduce_grad_more_local_pieces_than_the_cache(R, P):
     home = normal_bf16((E, P), seed=17, stream=12)
     got = _reduce(cfg, arena, rep, home, P)
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
     assert np.array_equal(got[1:], home[1:])  # experts without replicas untouched
 
 
@@ -291,8 +296,7 @@ def test_dispatch_backward_matches_oracle(shape):
     if ref.size == 0:
         assert got.size == 0
         return
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
 
 
 def test_dispatch_backward_is_adjoint_on_gpu():
@@ -421,9 +425,7 @@ def test_chained_calls_without_host_syncs():
     ref_home = oracle.reduce_grad(ocfg, ot, ref_rep, home0)
     ref_recv2 = oracle.dispatch(ocfg, ot2["slot_of"], ref_out)
 
-    def close(got, ref):  # fp32-accumulated results: the tolerance of the other data tests
-        assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-        assert (got == ref).mean() >= 0.999
+    close = _exact  # fp32-accumulated results: the bar of the other data tests
 
     assert np.array_equal(to_np(rep_w).reshape(R, cfg.budget, P), ref_rep)  # copies: bit-exact
     close(to_np(out), ref_out)
@@ -457,5 +459,4 @@ def test_reduce_grad_forced_timeout_reports_status_and_context_stays_usable():
         me.moonep_debug_set_wait(me.DEFAULT_WAIT_NS, 0)
     got = _reduce(cfg, arena, rep, home, P)
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
-    assert rel_err(bf16_bits_to_f32(got), bf16_bits_to_f32(ref)) <= TOL
-    assert (got == ref).mean() >= 0.999
+    _exact(got, ref)
