@@ -38,6 +38,7 @@ constexpr size_t kAlignBytes = 256;
 struct Dims {
   int64_t R, E, K, S, H, B, A, L, SK, N, NvS, NCMAX, PMAX;  // NCMAX: most plan chunks (512 pairs each)
   int mode;
+  uint32_t magicL;  // ceil(2^32 / L) for L > 1: e / L == __umulhi(e, magicL) for e < 2^22
 };
 
 __host__ __device__ inline int64_t nvs_of(int64_t S, int64_t K, int64_t E, int64_t A) {
@@ -63,6 +64,7 @@ inline bool make_dims(const moonep_config_t *c, Dims *d) {
   if (d->N >= (int64_t(1) << 31) || d->R * d->NvS >= (int64_t(1) << 31)) return false;
   d->NCMAX = d->N > 0 ? (d->N + kPlanThreads - 1) / kPlanThreads : 1;
   d->PMAX = d->E + d->R;
+  d->magicL = d->L > 1 ? (uint32_t)(0xFFFFFFFFu / (uint32_t)d->L) + 1u : 0u;
   return true;
 }
 
@@ -162,6 +164,11 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
     if (lane >= o) v += n;
   }
   return v;
+}
+
+// home rank of expert e (e / L) without a division
+__device__ __forceinline__ int home_of(const Dims &d, int e) {
+  return d.L == 1 ? e : (int)__umulhi((unsigned)e, d.magicL);
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -86,17 +86,25 @@ __device__ __forceinline__ int ld_relaxed(const int32_t *p) {
   return v;
 }
 
-// Warp-wide bounded wait until flags[0, n) all equal v.  False on timeout.
-// Polls with relaxed loads (independent, so they overlap) and fences once after.
+// Warp-wide bounded wait until flags[0, n) all equal v.  False on timeout.  Each
+// lane issues the loads of its (up to 16) flags of a 512-flag block together, so a
+// polling round costs one L2 round trip; one fence once everything has arrived.
 __device__ bool warp_wait_all(const int32_t *flags, int64_t n, int v, long long limit_ns) {
   const int lane = threadIdx.x & 31;
   const unsigned long long t0 = now_ns();
   int64_t from = 0;  // flags before `from` are known to have arrived
   for (;;) {
+    int got[16];
+#pragma unroll
+    for (int j = 0; j < 16; j++) {
+      const int64_t c = from + j * 32 + lane;
+      got[j] = c < n ? ld_relaxed(flags + c) : v;
+    }
     bool mine = true;
-    for (int64_t c = from + lane; c < n && c < from + 1024; c += 32) mine &= ld_relaxed(flags + c) == v;
+#pragma unroll
+    for (int j = 0; j < 16; j++) mine &= got[j] == v;
     if (__all_sync(0xffffffffu, mine)) {
-      from += 1024;
+      from += 16 * 32;
       if (from >= n) {
         asm volatile("fence.acq_rel.gpu;" ::: "memory");
         return true;
@@ -104,7 +112,6 @@ __device__ bool warp_wait_all(const int32_t *flags, int64_t n, int v, long long 
       continue;
     }
     if ((long long)(now_ns() - t0) > limit_ns) return false;
-    __nanosleep(32);
   }
 }
 
@@ -204,6 +211,8 @@ __device__ void column_sums(const int32_t *hist, int E, int64_t nrows, int *out,
 // Histogram of chunk k and the stable rank of each of its pairs among the
 // chunk's pairs of the same expert.  Pair of (warp w, step j, lane l) is
 // k*ch + w*32*ppt + j*32 + l.  ev[j]: expert id, -1 bad id, -2 past the end.
+// kU16: the histogram row is written as uint16 (a chunk holds at most 8192 pairs).
+template <bool kU16>
 __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *wh,
                                             int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -248,7 +257,10 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
       wh[w * E + e] = acc;
       acc += v;
     }
-    a.hist[k * E + e] = acc;
+    if (kU16)
+      reinterpret_cast<uint16_t *>(a.hist)[k * E + e] = (uint16_t)acc;
+    else
+      a.hist[k * E + e] = acc;
   }
   __syncthreads();
 #pragma unroll
@@ -686,7 +698,7 @@ __device__ __forceinline__ bool wait_flag(const int32_t *flag, int v, long long 
   return true;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+__global__ void __launch_bounds__(kPlanThreads) plan_multichunk_kernel(PlanArgs a) {
   // launched with programmatic stream serialisation: wait here until the
   // kernel before it in the stream (the router's top-k, the previous layer)
   // has completed and its writes are visible
@@ -757,7 +769,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   int epoch = 0;
   bool have_epoch = false;
   for (int64_t k = wk; k < a.nc; k += W) {
-    const bool bad = __syncthreads_or(count_chunk(a, k, smem, ev, rk));
+    const bool bad = __syncthreads_or(count_chunk<false>(a, k, smem, ev, rk));
     if (!have_epoch) {
       if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
       __syncthreads();
@@ -884,25 +896,675 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   }
 }
 
-// Largest dynamic shared memory a launch of f may request on device dev (the
-// opt-in limit less the kernel's static shared memory); 0 on error.
-template <typename F>
-int max_dynamic_smem(F f, int dev) {
-  int optin = 0;
-  cudaFuncAttributes fa;
-  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-      cudaFuncGetAttributes(&fa, f) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return optin - (int)fa.sharedSizeBytes;
+// ============================================ one chunk per CTA, every CTA solves ===
+// plan_kernel: W CTAs, CTA k owns chunk k (W = number of chunks, all co-resident).
+//   count    stable ranks of the chunk's pairs and its histogram (count_chunk);
+//            the histogram is published with an arrival flag.
+//   gather   every CTA sums every chunk's histogram: the expert counts, and the
+//            counts of the chunks before its own (its pairs' base offsets).  A
+//            chunk is added as soon as its flag shows this launch's epoch.
+//   solve    every CTA solves the O(E + R) balance problem itself, in one warp
+//            (shuffle scans and shared memory, no block barriers).  All CTAs
+//            reach the same tables, so no CTA waits for another after the gather.
+//   place    each CTA places its own pairs straight from its shared memory.
+//   tables   each CTA writes its share of the user-facing plan tables.
+// One grid-wide exchange (the arrivals) per plan.
+struct FastSmem {
+  int *cnt, *base, *gcst, *kept, *ovf, *oend, *nst, *row0, *npc, *i0, *pid0, *eflag, *epos;  // [E]
+  int *load, *over, *def, *ridx, *ntot, *nseg, *rrank, *rbase, *rend, *rfirst, *rstart;  // [R]
+  int *pexp, *precv, *post, *plen, *pst, *prow, *pscan;  // [PMAX]
+  int *misc;     // [16]: 0 receivers, 1 pieces, 2 capacity, 3 gather state, 4 remote pieces
+  int *scratch;  // 20 * kPlanWarps: the areas of the block scans
+  int *tmp;      // per-warp histograms [16][E] while counting, then gather partials
+};
+
+enum FastMisc { M_NRECV = 0, M_NPIECE = 1, M_CAP = 2, M_STATE = 3, M_NREMOTE = 4 };
+
+__host__ __device__ inline size_t fast_tmp_ints(const Dims &d) {
+  const size_t hist = size_t(kPlanWarps) * d.E;
+  const size_t gather = 2 * size_t(8 * kPlanThreads > d.E ? 8 * kPlanThreads : d.E);
+  return hist > gather ? hist : gather;
 }
 
-size_t plan_smem_bytes(const Dims &d) {
+__host__ __device__ inline size_t fast_smem_ints(const Dims &d) {
+  return 13 * d.E + 11 * d.R + 7 * d.PMAX + 16 + 20 * kPlanWarps + 4 + fast_tmp_ints(d);
+}
+
+__device__ __forceinline__ FastSmem carve_fast(const Dims &d, int *s) {
+  const int E = (int)d.E, R = (int)d.R, PM = (int)d.PMAX;
+  FastSmem m;
+  int **ea[13] = {&m.cnt, &m.base, &m.gcst, &m.kept, &m.ovf, &m.oend, &m.nst, &m.row0, &m.npc,
+                  &m.i0, &m.pid0, &m.eflag, &m.epos};
+  for (int i = 0; i < 13; i++) { *ea[i] = s; s += E; }
+  int **ra[11] = {&m.load, &m.over, &m.def, &m.ridx, &m.ntot, &m.nseg, &m.rrank, &m.rbase,
+                  &m.rend, &m.rfirst, &m.rstart};
+  for (int i = 0; i < 11; i++) { *ra[i] = s; s += R; }
+  int **pa[7] = {&m.pexp, &m.precv, &m.post, &m.plen, &m.pst, &m.prow, &m.pscan};
+  for (int i = 0; i < 7; i++) { *pa[i] = s; s += PM; }
+  m.misc = s; s += 16;
+  m.scratch = s; s += 20 * kPlanWarps;
+  s = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(s) + 15) & ~uintptr_t(15));
+  m.tmp = s;
+  return m;
+}
+
+// Sums of every chunk's histogram (uint16 rows): m.cnt[e] over all chunks and m.base[e]
+// over the chunks before chunk k.  Warp 0 alone polls the arrival flags (every CTA polling
+// with every thread would pile thousands of loads per round onto the same few L2 lines);
+// once all chunks (and the test-only phantom arrivals) show this launch's epoch, all
+// threads load the rows together.  A row is U = E / V units of V counts (V = 8: one
+// 16-byte load); thread group g (G groups of U threads, or one group when U >
+// kPlanThreads) takes chunks g, g + G, ...  Returns the state bits (kStTimeout, kStBad).
+template <int V>
+__device__ int gather_all(const PlanArgs &a, int64_t k, int epoch, const FastSmem &m) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int E = (int)a.d.E;
+  const uint16_t *hist = reinterpret_cast<const uint16_t *>(a.hist);
+  if (tid < 32) {
+    const bool ok = warp_wait_all(a.arrive, a.nc + a.phantom, epoch, a.wait_ns);
+    if (lane == 0) m.misc[M_STATE] = ok ? 0 : kStTimeout;
+  }
+  __syncthreads();
+  if (m.misc[M_STATE]) return kStTimeout;
+  const int U = E / V;
+  const int gw = U < kPlanThreads ? U : kPlanThreads;  // threads per group
+  const int G = kPlanThreads / gw;
+  const int g = tid / gw, u0 = tid % gw;
+  const int NU = (U + gw - 1) / gw;                    // units per thread (1, or 2 when V == 1)
+  constexpr int QN = V == 8 ? 1 : 2;                   // E <= 1024: U <= 128 units of 8 counts
+  int tot[QN][V], pre[QN][V];
+#pragma unroll
+  for (int q = 0; q < QN; q++)
+#pragma unroll
+    for (int v = 0; v < V; v++) tot[q][v] = pre[q][v] = 0;
+  bool bad = false;
+  if (g < G) {
+    for (int64_t r0 = g; r0 < a.nc; r0 += 8LL * G) {
+      uint32_t vals[8][QN][V == 8 ? 4 : 1];
+#pragma unroll
+      for (int j = 0; j < 8; j++) {  // the batch's loads first, then the sums
+        const int64_t r = r0 + (int64_t)j * G;
+#pragma unroll
+        for (int q = 0; q < QN; q++) {
+          const int u = u0 + q * gw;
+          const bool in = r < a.nc && q < NU && u < U;
+          if constexpr (V == 8) {
+            const uint4 t = in ? __ldcg(reinterpret_cast<const uint4 *>(hist + r * E) + u)
+                               : make_uint4(0, 0, 0, 0);
+            vals[j][q][0] = t.x;
+            vals[j][q][1] = t.y;
+            vals[j][q][2] = t.z;
+            vals[j][q][3] = t.w;
+          } else {
+            vals[j][q][0] = in ? __ldcg(hist + r * E + u) : 0u;
+          }
+        }
+        if (u0 == 0 && r < a.nc) bad |= __ldcg(a.badmark + r) == epoch;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int64_t r = r0 + (int64_t)j * G;
+#pragma unroll
+        for (int q = 0; q < QN; q++)
+#pragma unroll
+          for (int v = 0; v < V; v++) {
+            const int c = V == 8 ? (int)((vals[j][q][v >> 1] >> ((v & 1) * 16)) & 0xffffu)
+                                 : (int)vals[j][q][0];
+            tot[q][v] += c;
+            if (r < k) pre[q][v] += c;
+          }
+      }
+    }
+  }
+  if (bad) atomicOr(&m.misc[M_STATE], kStBad);
+  // partial sums of the groups, then one thread per expert adds them up
+  int *ptot = m.tmp, *ppre = m.tmp + G * E;
+  if (g < G) {
+#pragma unroll
+    for (int q = 0; q < QN; q++) {
+      const int u = u0 + q * gw;
+      if (q >= NU || u >= U) break;
+#pragma unroll
+      for (int v = 0; v < V; v++) {
+        ptot[g * E + u * V + v] = tot[q][v];
+        ppre[g * E + u * V + v] = pre[q][v];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kPlanThreads) {
+    int t = 0, p = 0;
+    for (int q = 0; q < G; q++) {
+      t += ptot[q * E + e];
+      p += ppre[q * E + e];
+    }
+    m.cnt[e] = t;
+    m.base[e] = p;
+  }
+  __syncthreads();
+  return m.misc[M_STATE];
+}
+
+// first i in [0, n) with a[i] > v (n if none); a non-decreasing.  The steps depend only
+// on n (no data-dependent branches): the same trip count for every thread.
+__device__ __forceinline__ int upper_bound_bf(const int *a, int n, int v) {
+  if (n <= 0) return 0;
+  const int *base = a;
+  int len = n;
+  while (len > 1) {
+    const int half = len >> 1;
+    base = base[half] <= v ? base + half : base;
+    len -= half;
+  }
+  return (int)(base - a) + (*base <= v ? 1 : 0);
+}
+
+// Exclusive scan over the block of NA values per thread, in thread order, with the
+// totals: one barrier.  Each call passes its own scratch area (NA * kPlanWarps ints) so
+// that no second barrier is needed before the area is written again.
+template <int NA>
+__device__ __forceinline__ void block_scan(const int (&v)[NA], int (&ex)[NA], int (&tot)[NA],
+                                           int *scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc[NA];
+#pragma unroll
+  for (int k = 0; k < NA; k++) inc[k] = warp_incl_scan(v[k]);
+  if (lane == 31)
+#pragma unroll
+    for (int k = 0; k < NA; k++) scratch[k * kPlanWarps + warp] = inc[k];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < NA; k++) {
+    int off = 0, t = 0;
+#pragma unroll
+    for (int w = 0; w < kPlanWarps; w++) {
+      const int x = scratch[k * kPlanWarps + w];
+      off += w < warp ? x : 0;
+      t += x;
+    }
+    ex[k] = off + inc[k] - v[k];
+    tot[k] = t;
+  }
+}
+
+// Thread t's contiguous share [b, e) of n elements (n <= 4 * kPlanThreads).
+__device__ __forceinline__ void share_of(int n, int &b, int &e) {
+  const int per = (n + kPlanThreads - 1) / kPlanThreads;
+  b = min((int)threadIdx.x * per, n);
+  e = min(b + per, n);
+}
+
+// The balance problem, from m.cnt, by the whole block (the fixed rule of the plan; see
+// the file header): block scans over experts, ranks and pieces, one thread per element
+// in between.  Writes the solve state into shared memory; misc[M_CAP] != 0 if a rank
+// would pass NvS rows or the tables do not fit together (unreachable).
+__device__ void solve_fast(const Dims &d, const FastSmem &m) {
+  const int tid = threadIdx.x;
+  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, A = (int)d.A, B = (int)d.B;
+  const int SK = (int)d.SK, NvS = (int)d.NvS, N = (int)d.N, PM = (int)d.PMAX;
+  int *scr = m.scratch;  // 8 areas of 4 * kPlanWarps ints
+  int eb, ee, hb, he;
+  share_of(E, eb, ee);
+  share_of(R, hb, he);
+  // (1) global exclusive prefix of the expert counts
+  {
+    int v[1] = {0}, ex[1], tot[1];
+    for (int e = eb; e < ee; e++) v[0] += m.cnt[e];
+    block_scan<1>(v, ex, tot, scr);
+    int run = ex[0];
+    for (int e = eb; e < ee; e++) {
+      m.gcst[e] = run;
+      run += m.cnt[e];
+    }
+    if (tid == 0) {
+      m.misc[M_CAP] = 0;
+      m.misc[M_NREMOTE] = 0;
+    }
+  }
+  __syncthreads();
+  // (2) rank loads; overflow and deficit bases; the receivers (ranks below S*K) in rank order
+  int n_recv;
+  {
+    int v[3] = {0, 0, 0}, ex[3], tot[3];
+    for (int h = hb; h < he; h++) {
+      const int ld = ((h + 1) * L < E ? m.gcst[(h + 1) * L] : N) - m.gcst[h * L];
+      m.load[h] = ld;
+      v[0] += ld > SK ? ld - SK : 0;
+      v[1] += ld < SK ? SK - ld : 0;
+      v[2] += ld < SK ? 1 : 0;
+    }
+    block_scan<3>(v, ex, tot, scr + 4 * kPlanWarps);
+    int ov = ex[0], df = ex[1], rf = ex[2];
+    for (int h = hb; h < he; h++) {
+      const int ld = m.load[h];
+      const int o = ld > SK ? ld - SK : 0, dd = ld < SK ? SK - ld : 0;
+      m.over[h] = ov;
+      m.def[h] = df;
+      m.nseg[h] = L;
+      if (dd > 0) {
+        m.ridx[h] = rf;
+        m.rrank[rf] = h;
+        m.rbase[rf] = df;
+        m.rend[rf] = df + dd;
+        rf++;
+      } else {
+        m.ridx[h] = -1;
+      }
+      ov += o;
+      df += dd;
+    }
+    n_recv = tot[2];
+  }
+  __syncthreads();
+  // (3) per expert: rows kept at home, its range [oend - ovf, oend) of the overflow
+  //     stream, the receivers it reaches (one piece each); piece ids and padded kept rows
+  //     by one scan
+  int n_piece, padtot;
+  {
+    int v[2] = {0, 0}, ex[2], tot[2];
+    for (int e = eb; e < ee; e++) {
+      const int h = home_of(d, e);
+      const int c = m.cnt[e];
+      const int cl = m.gcst[e] - m.gcst[h * L];
+      int kept = SK - cl;
+      kept = kept < 0 ? 0 : (kept > c ? c : kept);
+      const int ovf = c - kept;
+      const int ost = m.over[h] + (cl > SK ? cl - SK : 0);
+      int npc = 0, i0 = 0;
+      if (ovf > 0 && n_recv > 0) {
+        i0 = upper_bound_bf(m.rend, n_recv, ost);
+        int i1 = upper_bound_bf(m.rend, n_recv, ost + ovf - 1);
+        if (i1 >= n_recv) i1 = n_recv - 1;
+        if (i0 < n_recv) npc = i1 - i0 + 1;
+      }
+      m.kept[e] = kept;
+      m.ovf[e] = ovf;
+      m.oend[e] = ost + ovf;
+      m.npc[e] = npc;
+      m.i0[e] = i0;
+      m.eflag[e] = 0;
+      v[0] += npc;
+      v[1] += A > 1 ? roundup_i(kept, A) : kept;
+    }
+    block_scan<2>(v, ex, tot, scr + 8 * kPlanWarps);
+    int rp = ex[0], rk = ex[1];
+    for (int e = eb; e < ee; e++) {
+      m.pid0[e] = rp;
+      rp += m.npc[e];
+      m.epos[e] = rk;  // global prefix of the padded kept rows
+      const int kept = m.kept[e];
+      rk += A > 1 ? roundup_i(kept, A) : kept;
+    }
+    n_piece = tot[0] < PM ? tot[0] : PM;  // pieces <= experts + receivers - 1 < PMAX
+    padtot = tot[1];
+  }
+  __syncthreads();
+  // (4) one task per thread: an expert's segment start and first row; a rank's native
+  //     rows; a piece's expert, receiver and range; a receiver's first piece and count
+  int bad = 0;
+  for (int t = tid; t < E + R + n_piece + n_recv; t += kPlanThreads) {
+    if (t < E) {
+      const int e = t, h = home_of(d, e);
+      const int nst = m.epos[e] - m.epos[h * L];
+      m.nst[e] = nst;
+      m.row0[e] = h * NvS + nst;
+    } else if (t < E + R) {
+      const int h = t - E;
+      m.ntot[h] = ((h + 1) * L < E ? m.epos[(h + 1) * L] : padtot) - m.epos[h * L];
+    } else if (t < E + R + n_piece) {
+      const int pid = t - E - R;
+      const int e = upper_bound_bf(m.pid0, E, pid) - 1;  // its expert: the last first-id <= pid
+      int i = m.i0[e] + (pid - m.pid0[e]);
+      if (e < 0 || i < 0 || i >= n_recv || pid - m.pid0[e] >= m.npc[e]) {
+        bad = 1;
+        i = 0;
+      }
+      const int ee2 = e < 0 ? 0 : e;
+      const int ost = m.oend[ee2] - m.ovf[ee2];
+      const int os = ost > m.rbase[i] ? ost : m.rbase[i];
+      const int oe = m.oend[ee2] < m.rend[i] ? m.oend[ee2] : m.rend[i];
+      m.pexp[pid] = ee2;
+      m.precv[pid] = i;
+      m.post[pid] = os;
+      m.plen[pid] = oe - os;
+      m.pscan[pid] = A > 1 ? roundup_i(oe - os, A) : oe - os;
+    } else {
+      const int i = t - E - R - n_piece;
+      const int ef = upper_bound_bf(m.oend, E, m.rbase[i]);
+      const int el = upper_bound_bf(m.oend, E, m.rend[i] - 1);
+      int first = ef < E ? m.pid0[ef] + (i - m.i0[ef]) : 0;
+      const int last = el < E ? m.pid0[el] + (i - m.i0[el]) : -1;
+      if (first < 0 || first > last || last >= n_piece || L + (last - first + 1) > E) {
+        bad = 1;
+        first = 0;
+      }
+      m.rfirst[i] = first;
+      m.nseg[m.rrank[i]] = L + (last - first + 1);
+    }
+  }
+  if (bad) atomicOr(&m.misc[M_CAP], 1);
+  __syncthreads();
+  // (5) alignment > 1: a piece's start is its receiver's native rows plus the padded
+  //     lengths of the receiver's earlier pieces (a scan over the pieces)
+  if (A > 1) {
+    int pb, pe;
+    share_of(n_piece, pb, pe);
+    int v[1] = {0}, ex[1], tot[1];
+    for (int pid = pb; pid < pe; pid++) v[0] += m.pscan[pid];
+    block_scan<1>(v, ex, tot, scr + 16 * kPlanWarps);
+    __syncthreads();  // every thread has read its values before they are overwritten
+    int run = ex[0];
+    for (int pid = pb; pid < pe; pid++) {
+      const int x = m.pscan[pid];
+      m.pscan[pid] = run;
+      run += x;
+    }
+    __syncthreads();
+  }
+  // (6) one piece per thread: its first row within the receiving rank (alignment 1: the
+  //     receiver's rows follow its native rows in overflow-stream order), capacity,
+  //     local-replica flags, remote pieces
+  int cap = 0, nrem = 0;
+  for (int pid = tid; pid < n_piece; pid += kPlanThreads) {
+    const int i = m.precv[pid], first = m.rfirst[i], dr = m.rrank[i];
+    if (pid < first) cap = 1;
+    const int st = A > 1 ? m.ntot[dr] + m.pscan[pid] - m.pscan[first]
+                         : m.ntot[dr] + (m.post[pid] - m.rbase[i]);
+    m.pst[pid] = st;
+    m.prow[pid] = dr * NvS + st;
+    if (st + m.plen[pid] > NvS) cap = 1;
+    if (pid - first < B) m.eflag[m.pexp[pid]] = 1;
+    else nrem++;
+  }
+  for (int h = tid; h < R; h += kPlanThreads)
+    if (m.ntot[h] > NvS) cap = 1;
+  if (cap) atomicOr(&m.misc[M_CAP], 1);
+  if (nrem) atomicAdd(&m.misc[M_NREMOTE], nrem);
+  if (tid == 0) {
+    m.misc[M_NRECV] = n_recv;
+    m.misc[M_NPIECE] = n_piece;
+  }
+  __syncthreads();
+}
+
+// Row of a pair at position pos of expert e's list (solve state in shared memory).
+__device__ __forceinline__ int fast_row(const FastSmem &m, int e, int pos) {
+  const int kept = m.kept[e];
+  if (pos < kept) return m.row0[e] + pos;
+  const int o = m.oend[e] - m.ovf[e] + (pos - kept);
+  int lo = m.pid0[e], hi = lo + m.npc[e] - 1;  // the last piece of e starting at or before o
+  if (hi < lo) return -1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.post[mid] <= o) lo = mid; else hi = mid - 1;
+  }
+  return m.prow[lo] + (o - m.post[lo]);
+}
+
+// True if row `row` of rank h holds a pair (inside a segment), false for padding.
+__device__ __forceinline__ bool fast_row_used(const Dims &d, const FastSmem &m, int h, int row) {
+  const int L = (int)d.L;
+  if (row < m.ntot[h]) {  // native segments: the last expert starting at or before row
+    int lo = h * L, hi = h * L + L - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (m.nst[mid] <= row) lo = mid; else hi = mid - 1;
+    }
+    return row < m.nst[lo] + m.kept[lo];
+  }
+  const int i = m.ridx[h];
+  if (i < 0) return false;
+  int lo = m.rfirst[i], hi = lo + (m.nseg[h] - L) - 1;
+  if (hi < lo) return false;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m.pst[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  return m.pst[lo] <= row && row < m.pst[lo] + m.plen[lo];
+}
+
+// The user-facing tables, shared over the CTAs (every CTA holds the whole solve).
+__device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
+  const Dims &d = a.d;
+  const PlanPtrs &P = a.P;
+  const int tid = threadIdx.x;
+  const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
+  const int n_piece = min(m.misc[M_NPIECE], (int)d.PMAX);
+  const int64_t gt = (int64_t)blockIdx.x * kPlanThreads + tid;
+  const int64_t stride = (int64_t)gridDim.x * kPlanThreads;
+  for (int64_t e = gt; e < E; e += stride) {
+    const int h = (int)e / L;
+    const int64_t si = (int64_t)h * E + (e - (int64_t)h * L);
+    P.f[F_EXPERT_COUNT][e] = m.cnt[e];
+    P.f[F_EXP_PIECE_BEGIN][e] = m.pid0[e];
+    P.f[F_EXP_PIECE_END][e] = m.pid0[e] + m.npc[e];
+    P.f[F_SEG_EXPERT][si] = (int)e;
+    P.f[F_SEG_START][si] = m.nst[e];
+    P.f[F_SEG_LEN][si] = m.kept[e];
+    P.f[F_SEG_KIND][si] = MOONEP_SEG_NATIVE;
+    P.f[F_SEG_WSLOT][si] = -1;
+  }
+  for (int64_t pid = gt; pid < n_piece; pid += stride) {
+    const int i = m.precv[pid], dr = m.rrank[i], j = (int)pid - m.rfirst[i], e = m.pexp[pid];
+    const int ws = j < B ? j : -1;
+    P.f[F_PIECE_EXPERT][pid] = e;
+    P.f[F_PIECE_RANK][pid] = dr;
+    P.f[F_PIECE_START][pid] = m.pst[pid];
+    P.f[F_PIECE_LEN][pid] = m.plen[pid];
+    P.f[F_PIECE_WSLOT][pid] = ws;
+    P.f[F_PIECE_OSTART][pid] = m.post[pid];
+    if (j >= 0 && L + j < E) {
+      const int64_t sj = (int64_t)dr * E + L + j;
+      P.f[F_SEG_EXPERT][sj] = e;
+      P.f[F_SEG_START][sj] = m.pst[pid];
+      P.f[F_SEG_LEN][sj] = m.plen[pid];
+      P.f[F_SEG_KIND][sj] = ws >= 0 ? MOONEP_SEG_REPLICA : MOONEP_SEG_REMOTE;
+      P.f[F_SEG_WSLOT][sj] = ws;
+    }
+    if (ws >= 0) P.f[F_REP_EXPERT][(int64_t)dr * B + j] = e;
+  }
+  for (int64_t h = gt; h < R; h += stride) {
+    const int ld = m.load[h];
+    P.f[F_RANK_LOAD][h] = ld;
+    P.f[F_OVERFLOW][h] = ld > SK ? ld - SK : 0;
+    P.f[F_DEFICIT][h] = ld < SK ? SK - ld : 0;
+    P.f[F_N_SEG][h] = m.nseg[h];
+  }
+  for (int64_t q = gt; q < (int64_t)R * E; q += stride) {  // unused segment entries
+    const int h = (int)(q / E), i = (int)(q % E);
+    if (i >= m.nseg[h]) {
+      P.f[F_SEG_EXPERT][q] = -1;
+      P.f[F_SEG_START][q] = 0;
+      P.f[F_SEG_LEN][q] = 0;
+      P.f[F_SEG_KIND][q] = -1;
+      P.f[F_SEG_WSLOT][q] = -1;
+    }
+  }
+  for (int64_t q = gt; q < (int64_t)R * B; q += stride) {  // free replica weight slots
+    const int h = (int)(q / B), j = (int)(q % B);
+    if (j >= m.nseg[h] - L) P.f[F_REP_EXPERT][q] = -1;
+  }
+  if (d.A > 1) {  // padding rows hold no pair
+    int32_t *slot_src = P.f[F_SLOT_SRC];
+    for (int64_t q = gt; q < d.R * d.NvS; q += stride)
+      if (!fast_row_used(d, m, (int)(q / d.NvS), (int)(q % d.NvS))) slot_src[q] = -1;
+  }
+  if (blockIdx.x == gridDim.x - 1) {  // the last chunk is the smallest: this CTA adds the rest
+    for (int e = tid; e < E; e += kPlanThreads) m.epos[e] = m.eflag[e];
+    int *arr[1] = {m.epos};
+    int tot[1];
+    __syncthreads();
+    block_excl_scan<1>(arr, E, m.scratch, tot);
+    for (int e = tid; e < E; e += kPlanThreads)
+      if (m.eflag[e]) P.f[F_REPLICATED][m.epos[e]] = e;
+    if (tid == 0) {
+      const int n_remote = m.misc[M_NREMOTE];
+      int32_t *sc = P.f[F_SCALARS];
+      sc[S_N_PIECE] = n_piece;
+      sc[S_N_REMOTE] = n_remote;
+      sc[S_N_LOCAL] = n_piece - n_remote;
+      sc[S_N_REPLICATED] = tot[0];
+      sc[S_BAD] = 0;
+      sc[5] = sc[6] = sc[7] = 0;
+      if (d.mode == MOONEP_MODE_TRAIN && n_remote > 0) set_status(a.status, MOONEP_DEV_BUDGET);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  // launched with programmatic stream serialisation: wait here until the kernel
+  // before it in the stream (the router's top-k, the previous layer) has completed
+  // and its writes are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ __align__(16) int smem[];
+  __shared__ int s_epoch;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Dims &d = a.d;
+  const int64_t k = blockIdx.x;  // this CTA's chunk
+  const FastSmem m = carve_fast(d, smem);
+  int32_t *gen = a.sync + kSyncGen;
+  // the generation word: needed only when the chunk is published, so its load
+  // overlaps the counting
+  int gen_v = 0;
+  if (tid == 0) gen_v = *((volatile int32_t *)gen);
+  int ev[kPairsPerThread], rk[kPairsPerThread];
+  const bool bad = __syncthreads_or(count_chunk<true>(a, k, m.tmp, ev, rk));
+  if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
+  __syncthreads();
+  const int epoch = s_epoch;
+  if (tid == 0) {
+    if (bad) set_status(a.status, MOONEP_DEV_BAD_EXPERT_ID);
+    a.badmark[k] = bad ? epoch : ~epoch;
+    // the histogram row was written by every thread before the barriers above; the
+    // release store orders all of it (barrier, then release: cumulative) before the flag
+    st_release(a.arrive + k, epoch);
+  }
+  int st = (d.E & 7) == 0 ? gather_all<8>(a, k, epoch, m) : gather_all<1>(a, k, epoch, m);
+  // every CTA has arrived, so every CTA has read the generation word; a bad id
+  // does not stop this, the next launch must get a new epoch in any case
+  if (k == 0 && tid == 0) *((volatile int32_t *)gen) = epoch;
+  if (st == 0) {
+    solve_fast(d, m);
+    if (m.misc[M_CAP]) st = kStCapacity;
+  }
+  int32_t *slot_of = a.P.f[F_SLOT_OF];
+  if (st) {  // an invalid plan: no pair has a slot, no row a pair
+    const int64_t p0 = k * a.ch, p1 = (k + 1) * a.ch < d.N ? (k + 1) * a.ch : d.N;
+    for (int64_t p = p0 + tid; p < p1; p += kPlanThreads) slot_of[p] = -1;
+    int32_t *slot_src = a.P.f[F_SLOT_SRC];
+    for (int64_t q = k * kPlanThreads + tid; q < d.R * d.NvS; q += (int64_t)gridDim.x * kPlanThreads)
+      slot_src[q] = -1;
+    if (tid == 0) {
+      if (st & kStTimeout) set_status(a.status, MOONEP_DEV_TIMEOUT);
+      if (k == 0) {
+        if (st & kStCapacity) set_status(a.status, MOONEP_DEV_CAPACITY);
+        int32_t *sc = a.P.f[F_SCALARS];
+        for (int i = 0; i < 8; i++) sc[i] = 0;
+        sc[S_BAD] = st;
+      }
+    }
+    return;
+  }
+  // place this chunk's pairs
+  {
+    int32_t *slot_src = a.P.f[F_SLOT_SRC];
+    const int64_t nrows = d.R * d.NvS;
+    const int64_t base = k * a.ch + (int64_t)warp * 32 * a.ppt;
+#pragma unroll
+    for (int j = 0; j < kPairsPerThread; j++) {
+      if (j >= a.ppt) break;
+      const int64_t p = base + j * 32 + lane;
+      if (p >= d.N) continue;
+      const int e = ev[j];
+      int row = e >= 0 ? fast_row(m, e, m.base[e] + rk[j]) : -1;
+      if (row < 0 || row >= nrows) row = -1;  // unreachable for a consistent plan
+      slot_of[p] = row;
+      if (row >= 0) slot_src[row] = (int32_t)p;
+    }
+  }
+  fast_tables(a, m);
+}
+
+size_t plan_multichunk_smem_bytes(const Dims &d) {
   const size_t worker = std::max<size_t>(size_t(kPlanWarps) * d.E,
                                          6 * d.E + 2 * d.PMAX + 4 + 4 * kPlanThreads);
   const size_t solver = solve_smem_ints(d);
   return std::max(worker, solver) * sizeof(int) + 16;
+}
+
+size_t plan_smem_bytes(const Dims &d) { return fast_smem_ints(d) * sizeof(int) + 16; }
+
+// Host-side launch facts of the two plan kernels, cached per device for the
+// context they were taken in (a kernel's dynamic shared memory limit is a
+// per-context attribute): SM count, the opt-in shared memory limit, and
+// co-resident CTAs per SM for the dynamic shared memory sizes seen so far.
+struct KernelLaunchInfo {
+  int limit = 0;          // largest dynamic shared memory a launch may request
+  bool attr_set = false;  // that limit has been set on the kernel in this context
+  size_t occ_smem[8] = {};
+  int occ_ctas[8] = {};
+  int occ_n = 0;
+};
+struct DeviceLaunchInfo {
+  unsigned long long ctx = 0;
+  int sms = 0;
+  KernelLaunchInfo k[2];  // 0: plan_kernel, 1: plan_multichunk_kernel
+};
+std::mutex g_launch_mu;
+DeviceLaunchInfo g_launch[kMaxDevices];
+
+// Co-resident CTAs per SM of kernel `which` with `smem` bytes of dynamic shared
+// memory (the kernel's limit raised first when past 48 KB); 0 if it does not
+// fit, -1 on a CUDA error.  *sms receives the SM count.
+template <typename F>
+int plan_ctas_per_sm(F f, int which, int dev, size_t smem, int *sms) {
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  DeviceLaunchInfo &di = g_launch[dev];
+  if (ctx == 0 || di.ctx != ctx) {  // first call in this context (or no context id)
+    di = DeviceLaunchInfo();
+    di.ctx = ctx;
+  }
+  if (di.sms == 0 && (cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev) !=
+                          cudaSuccess || di.sms <= 0)) {
+    cudaGetLastError();
+    di.sms = 0;
+    return -1;
+  }
+  *sms = di.sms;
+  KernelLaunchInfo &ki = di.k[which];
+  if (ki.limit == 0) {
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, f) != cudaSuccess) {
+      cudaGetLastError();
+      return -1;
+    }
+    ki.limit = optin - (int)fa.sharedSizeBytes;
+    if (ki.limit <= 0) return -1;
+  }
+  if (smem > size_t(ki.limit)) return 0;
+  // the device's whole limit, so concurrent callers with other configs never lower
+  // it under each other
+  if (smem > 48 * 1024 && !ki.attr_set) {
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, ki.limit) != cudaSuccess) {
+      cudaGetLastError();
+      return -1;
+    }
+    ki.attr_set = true;
+  }
+  for (int i = 0; i < ki.occ_n; i++)
+    if (ki.occ_smem[i] == smem) return ki.occ_ctas[i];
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, f, kPlanThreads, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  const int slot = ki.occ_n < 8 ? ki.occ_n++ : int(smem % 8);
+  ki.occ_smem[slot] = smem;
+  ki.occ_ctas[slot] = per_sm;
+  return per_sm;
 }
 
 }  // namespace
@@ -972,35 +1634,50 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOONEP_ERR_CUDA;
-  const size_t smem = plan_smem_bytes(d);
-  const int limit = max_dynamic_smem(plan_kernel, dev);
-  if (limit <= 0) return MOONEP_ERR_CUDA;
-  if (smem > size_t(limit)) return MOONEP_ERR_UNSUPPORTED;
-  // the device's whole limit, so concurrent callers with other configs never
-  // lower it under each other
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) !=
-          cudaSuccess)
-    return MOONEP_ERR_CUDA;
-  // co-resident CTAs: a cooperative launch guarantees they run at the same time
-  int sms = 0, per_sm = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, kPlanThreads, smem) !=
-          cudaSuccess)
-    return MOONEP_ERR_CUDA;
-  const int64_t coresident = (int64_t)sms * per_sm;
-  if (coresident < 2) return MOONEP_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) return MOONEP_ERR_UNSUPPORTED;
 
+  // one chunk per CTA when the chunks fit on the co-resident CTAs: pairs spread
+  // over them, 512..8192 pairs a chunk (a cooperative launch guarantees that the
+  // CTAs run at the same time)
+  int sms = 0;
+  const size_t smem = plan_smem_bytes(d);
+  const int per_sm = plan_ctas_per_sm(plan_kernel, 0, dev, smem, &sms);
+  if (per_sm < 0) return MOONEP_ERR_CUDA;
   PlanArgs a;
   a.d = d;
-  // chunk size: spread the pairs over every co-resident worker, 512..8192 pairs
-  const int64_t wmax = coresident - 1;
-  int64_t ppt = (d.N + wmax * kPlanThreads - 1) / (wmax * kPlanThreads);
-  ppt = ppt < 1 ? 1 : (ppt > kPairsPerThread ? kPairsPerThread : ppt);
-  a.ppt = (int)ppt;
-  a.ch = ppt * kPlanThreads;
-  a.nc = d.N > 0 ? (d.N + a.ch - 1) / a.ch : 1;
-  a.workers = (int)(a.nc < wmax ? a.nc : wmax);
+  bool one_chunk_per_cta = false;
+  void (*kernel)(PlanArgs) = plan_kernel;
+  size_t kernel_smem = smem;
+  if (per_sm > 0) {
+    const int64_t coresident = (int64_t)sms * per_sm;
+    int64_t ppt = (d.N + coresident * kPlanThreads - 1) / (coresident * kPlanThreads);
+    ppt = ppt < 1 ? 1 : ppt;
+    if (ppt <= kPairsPerThread) {
+      one_chunk_per_cta = true;
+      a.ppt = (int)ppt;
+      a.ch = ppt * kPlanThreads;
+      a.nc = d.N > 0 ? (d.N + a.ch - 1) / a.ch : 1;
+      a.workers = (int)a.nc;
+    }
+  }
+  if (!one_chunk_per_cta) {
+    // chunks outnumber the co-resident CTAs: one solving CTA, workers with
+    // several chunks each
+    kernel = plan_multichunk_kernel;
+    kernel_smem = plan_multichunk_smem_bytes(d);
+    const int ms = plan_ctas_per_sm(plan_multichunk_kernel, 1, dev, kernel_smem, &sms);
+    if (ms < 0) return MOONEP_ERR_CUDA;
+    if (ms == 0) return MOONEP_ERR_UNSUPPORTED;
+    const int64_t coresident = (int64_t)sms * ms;
+    if (coresident < 2) return MOONEP_ERR_UNSUPPORTED;
+    const int64_t wmax = coresident - 1;
+    int64_t ppt = (d.N + wmax * kPlanThreads - 1) / (wmax * kPlanThreads);
+    ppt = ppt < 1 ? 1 : (ppt > kPairsPerThread ? kPairsPerThread : ppt);
+    a.ppt = (int)ppt;
+    a.ch = ppt * kPlanThreads;
+    a.nc = d.N > 0 ? (d.N + a.ch - 1) / a.ch : 1;
+    a.workers = (int)(a.nc < wmax ? a.nc : wmax);
+  }
   if (a.nc > d.NCMAX) return MOONEP_ERR_UNSUPPORTED;  // cannot happen: chunks >= 512 pairs
   a.idx = topk_idx;
   a.P = plan_ptrs(d, plan_arena);
@@ -1020,9 +1697,9 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   a.phantom = g_phantom_arrivals.load(std::memory_order_relaxed);
 
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3((unsigned)(a.workers + 1));
+  lc.gridDim = dim3((unsigned)(one_chunk_per_cta ? a.nc : a.workers + 1));
   lc.blockDim = dim3(kPlanThreads);
-  lc.dynamicSmemBytes = smem;
+  lc.dynamicSmemBytes = kernel_smem;
   lc.stream = to_cuda(stream);
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -1033,12 +1710,12 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   // programmatic dependent launch hides the launch gap after the previous
   // kernel; without it (a runtime that refuses the pair) the launch is plain
   lc.numAttrs = g_plan_pdl.load(std::memory_order_relaxed) ? 2 : 1;
-  if (cudaLaunchKernelEx(&lc, plan_kernel, a) == cudaSuccess) return MOONEP_OK;
+  if (cudaLaunchKernelEx(&lc, kernel, a) == cudaSuccess) return MOONEP_OK;
   cudaGetLastError();
   if (lc.numAttrs == 2) {
     g_plan_pdl.store(false);
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, plan_kernel, a) == cudaSuccess) return MOONEP_OK;
+    if (cudaLaunchKernelEx(&lc, kernel, a) == cudaSuccess) return MOONEP_OK;
     cudaGetLastError();
   }
   return MOONEP_ERR_CUDA;
