@@ -3,23 +3,28 @@
 // duplicated onto underloaded ranks within a replica-slot budget;
 // "MoonshotAI/MoonEP 딥다이브" §4 pattern 1: planned once per layer, reused).
 //
-// One cooperative kernel: CTA 0 solves, CTAs 1..W are workers.
-//   workers  take chunks of 512*ppt (rank, token, k) pairs (ppt <= 16, sized so
-//            that all SMs share the work).  Warp-private per-expert counters in
-//            shared memory give every pair its stable rank among the chunk's
-//            pairs of the same expert (lanes with equal ids are found with a
-//            shuffle-built peer mask: a hot expert costs one counter update per
-//            warp step, no atomics); the chunk histogram is published with an
-//            arrival flag.  While CTA 0 solves, each worker sums the histograms
-//            of the chunks before its own into its chunk's base offsets.
-//   CTA 0    waits for every arrival, sums the histograms into expert counts and
-//            solves the O(E + R) balance problem in shared memory.  It publishes
-//            the tables placement needs first (done flag), then writes the
-//            remaining plan tables while the workers place.
-//   workers  wait for the done flag and place their pairs: position in the
-//            expert's list = chunk base + stable rank; the first kept_e
-//            positions stay in the home segment, the rest map through the
-//            expert's pieces.
+// The rule (pairs of an expert in (rank, token, k) order; each home rank keeps the
+// first S*K entries of its experts' lists in ascending expert order; the rest, over
+// ranks ascending, fill the underloaded ranks in ascending order; pieces, budget and
+// alignment as in include/moonep.h) is computed by one cooperative kernel:
+//
+// plan_kernel (chunks <= co-resident CTAs): CTA k owns chunk k of 512*ppt pairs.
+//   count    warp-private per-expert counters in shared memory give every pair its
+//            stable rank among the chunk's pairs of the same expert (lanes with
+//            equal ids found with match.any: a hot expert costs one counter update
+//            per warp step, no atomics); the chunk histogram is published as a
+//            uint16 row with one release store of an arrival flag.
+//   gather   once every flag shows this launch's epoch (warp 0 polls), each CTA
+//            sums all rows: the expert counts, and the counts of the chunks
+//            before its own (its pairs' base offsets).
+//   solve    each CTA solves the O(E + R) problem itself with block scans; all
+//            CTAs reach the same tables, so nobody waits for anybody again.
+//   place    each CTA places its own pairs straight from its shared memory.
+//   tables   each CTA writes its share of the user-facing plan tables.
+// plan_multichunk_kernel (larger batches): CTA 0 solves, CTAs 1..W are workers
+//            with several chunks each; workers keep stable ranks in the workspace,
+//            the solver turns the histograms into per-chunk bases and publishes the
+//            placement tables with a done flag.
 // Flags carry a per-launch epoch derived from a generation word on the device,
 // so graph replays and reused workspaces need no memset; every wait is bounded
 // in time and reports MOONEP_DEV_TIMEOUT instead of hanging.
