@@ -491,16 +491,31 @@ def compact_sweep(layer, seeds, steps, warmup, targets=SWEEP_MAXVIO):
             "peak_GBs": peak, "rows": rows, "clocks": merge_clocks(clocks)}
 
 
+def fused_pass(layer, steps, warmup):
+    """The same forward layer as one launch (moonep_fused_forward: plan, dispatch and the
+    identity expert's combine): overlapped layer time and per-call event time."""
+    me, c = layer.me, layer.cfg
+    ops = [("fused", lambda: me.moonep_fused_forward(c, layer.idx, layer.gates, layer.x, layer.arena,
+                                                     layer.ws, layer.recv, layer.out, layer.status))]
+    total_ms, per, clocks, st = time_steps(layer, steps, warmup, ops=ops)
+    return {"fused_layer_us": 1e3 * total_ms / steps,
+            "fused_layer_us_kernel_events": 1e3 * statistics.median(per["fused"]),
+            "fused_status": st}, clocks
+
+
 def decode_runs(device, steps, warmup, maxvios=(1.0, 20.0), seed=0):
-    """The 64-rank inference workload: plan + dispatch + combine µs per maxvio."""
+    """The 64-rank inference workload: plan + dispatch + combine µs per maxvio, as three
+    calls and as the one-launch fused layer."""
     w = WORKLOADS[DECODE_WORKLOAD]
     layer = Layer(w, maxvios[0], seed, device, with_backward=False, host_inputs=False)
     out, clocks = [], []
     for mv in maxvios:
         layer.set_routing(mv, seed)
         r, c = forward_pass(layer, steps, warmup)
+        fr, fc = fused_pass(layer, steps, warmup)
+        r.update(fr)
         out.append(r)
-        clocks.append(c)
+        clocks += [c, fc]
     b = layer.bytes(forward_only=True)
     res = {"workload": w.name, "seed": seed, "steps": steps,
            "bytes_dispatch_combine": b["dispatch"] + b["combine"],

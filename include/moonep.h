@@ -11,6 +11,7 @@
  *   moonep_reduce_grad       fold replica-expert gradients into their home experts
  *   moonep_dispatch_backward gradient of dispatch (sum of a token's K slot gradients)
  *   moonep_prefetch_weight   copy duplicated experts' weights into replica slots
+ *   moonep_fused_forward     plan + dispatch + combine of the identity expert in one launch
  *
  * Conventions shared by every call:
  *   - Ownership: the caller allocates and frees every buffer (device memory
@@ -290,6 +291,29 @@ MOONEP_API moonep_status_t moonep_combine_via_buffer(const moonep_config_t *cfg,
                                                      const float *gates, const int32_t *comm_index,
                                                      uint16_t *comm, uint16_t *out,
                                                      int32_t *dev_status, moonep_stream_t stream);
+
+/* The forward layer of the identity expert in one launch, for small batches where
+ * launch and hand-off latency matter (the decode path: "Moonshot AI Open-Sources
+ * MoonEP", replica-slot paragraph, inference with a few replica slots): moonep_plan,
+ * then moonep_dispatch of x into recv, then moonep_combine of y = recv, with the same
+ * results bit for bit as those three calls.  Each CTA of the plan's one-chunk-per-CTA
+ * launch dispatches and combines the tokens of its own chunk right after placing
+ * them: under the identity expert a token's combine reads only rows that the same
+ * CTA has just written, so no second grid-wide exchange is needed.  (With a real
+ * expert between dispatch and combine this call does not apply.)
+ *   topk_idx, gates, x, plan_arena, workspace, dev_status: as for moonep_plan /
+ *   moonep_dispatch / moonep_combine; recv bf16 [R*NvS, H] (padding rows untouched);
+ *   out bf16 [R*S, H].  The plan tables are complete when the launch ends.
+ * MOONEP_ERR_UNSUPPORTED when K does not divide 512 or K > 8 (a chunk must hold whole
+ * tokens), H % 8 != 0, x / recv / out not 16-byte aligned, or the batch needs more
+ * chunks than co-resident CTAs (more than about 148 * 8192 pairs): use the separate
+ * calls then.  A plan that fails (bad expert id, timeout) dispatches nothing and
+ * writes zero output rows, as the separate calls would. */
+MOONEP_API moonep_status_t moonep_fused_forward(const moonep_config_t *cfg, const int32_t *topk_idx,
+                                                const float *gates, const uint16_t *x,
+                                                void *plan_arena, void *workspace, uint16_t *recv,
+                                                uint16_t *out, int32_t *dev_status,
+                                                moonep_stream_t stream);
 
 /* Static description of a status code. */
 MOONEP_API const char *moonep_status_string(moonep_status_t status);

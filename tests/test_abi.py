@@ -154,3 +154,26 @@ def test_debug_wait_knob_validates_arguments():
     assert me._lib.moonep_debug_set_wait(1000, 33) == me.ERR_INVALID_ARG
     assert me._lib.moonep_debug_set_wait(1000, -1) == me.ERR_INVALID_ARG
     assert me._lib.moonep_debug_set_wait(me.DEFAULT_WAIT_NS, 0) == me.OK
+
+
+def test_fused_forward_checks_arguments_on_host():
+    """The fused layer refuses, before any CUDA call, what its one-launch design cannot
+    do: K not dividing 512 or above 8, rows that are not 16-byte multiples, misaligned
+    rows; and null pointers."""
+    L = me._lib
+    base = 1 << 30
+    ok = me.Config(R=2, E=8, K=2, S=4, H=16, budget=2)
+    cp = ctypes.byref(ok)
+    assert L.moonep_fused_forward(cp, None, base, base, base, base, base, base, base, 0) == \
+        me.ERR_INVALID_ARG
+    assert L.moonep_fused_forward(cp, base, base, base, base, base, base, base, None, 0) == \
+        me.ERR_INVALID_ARG
+    assert L.moonep_fused_forward(cp, base, base, base, base + 16, base, base, base, base, 0) == \
+        me.ERR_INVALID_ARG
+    assert L.moonep_fused_forward(cp, base, base, base + 2, base, base, base, base, base, 0) == \
+        me.ERR_UNSUPPORTED
+    for bad in (me.Config(R=2, E=8, K=3, S=4, H=16, budget=2),
+                me.Config(R=2, E=32, K=16, S=4, H=16, budget=2),
+                me.Config(R=2, E=8, K=2, S=4, H=12, budget=2)):
+        assert L.moonep_fused_forward(ctypes.byref(bad), base, base, base, base, base, base, base,
+                                      base, 0) == me.ERR_UNSUPPORTED

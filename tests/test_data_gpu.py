@@ -460,3 +460,27 @@ def test_reduce_grad_forced_timeout_reports_status_and_context_stays_usable():
     got = _reduce(cfg, arena, rep, home, P)
     ref = oracle.reduce_grad(ocfg, ot, rep, home)
     _exact(got, ref)
+
+
+@pytest.mark.parametrize("R,E,K,S,B,P,mv", [(8, 384, 8, 512, 48, 4096 + 8, 20.0),
+                                             (8, 256, 8, 256, 32, 24, 0.2),
+                                             (64, 256, 8, 64, 4, 8192, 20.0)])
+def test_replica_rows_of_ragged_lengths(R, E, K, S, B, P, mv):
+    """reduce_grad and prefetch_weight move expert rows in 8 KB units: rows of one short
+    unit, of one full unit plus 16 bytes, and many experts with few units each must all
+    come out exact."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=mv, seed=31, budget=B, mode=1)
+    assert int(ot["n_piece"][0]) > 0
+    rep = normal_bf16((R, B, P), seed=31, stream=11)
+    home = normal_bf16((E, P), seed=31, stream=12)
+    _exact(_reduce(cfg, arena, rep, home, P), oracle.reduce_grad(ocfg, ot, rep, home))
+    w = normal_bf16((E, P), seed=32, stream=14)
+    before = normal_bf16((R, B, P), seed=33, stream=15)
+    out = to_dev(before)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    me.moonep_prefetch_weight(cfg, arena, to_dev(w), out, P, status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert np.array_equal(to_np(out), oracle.prefetch_weight(ocfg, ot, w, before))

@@ -20,6 +20,7 @@ The functions keep the C names::
     moonep_prefetch_weight(cfg, plan_arena, weights, rep_weights, W, dev_status, stream=None)
     moonep_dispatch_via_buffer(cfg, plan_arena, x, comm, comm_index, recv, dev_status, stream=None)
     moonep_combine_via_buffer(cfg, plan_arena, y, gates, comm_index, comm, out, dev_status, stream=None)
+    moonep_fused_forward(cfg, topk_idx, gates, x, plan_arena, workspace, recv, out, dev_status, stream=None)
 
 Tensor arguments are device tensors (bf16 tensors may be ``torch.bfloat16``
 or ``int16``/``uint16`` views); raw integer device addresses are accepted too.
@@ -139,6 +140,8 @@ _lib.moonep_dispatch_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _
 _lib.moonep_dispatch_via_buffer.restype = _ST
 _lib.moonep_combine_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_combine_via_buffer.restype = _ST
+_lib.moonep_fused_forward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
+_lib.moonep_fused_forward.restype = _ST
 _lib.moonep_status_string.argtypes = [_ST]
 _lib.moonep_status_string.restype = ctypes.c_char_p
 
@@ -289,6 +292,13 @@ def moonep_combine_via_buffer(cfg: Config, plan_arena, y, gates, comm_index, com
     _check("moonep_combine_via_buffer", _lib.moonep_combine_via_buffer(
         ctypes.byref(cfg), _ptr(plan_arena), _ptr(y), _ptr(gates), _ptr(comm_index), _ptr(comm),
         _ptr(out), _ptr(dev_status), _stream(stream)))
+
+
+def moonep_fused_forward(cfg: Config, topk_idx, gates, x, plan_arena, workspace, recv, out,
+                         dev_status, stream=None) -> None:
+    _check("moonep_fused_forward", _lib.moonep_fused_forward(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(gates), _ptr(x), _ptr(plan_arena), _ptr(workspace),
+        _ptr(recv), _ptr(out), _ptr(dev_status), _stream(stream)))
 
 
 # ---------------------------------------------------------- allocation help ---

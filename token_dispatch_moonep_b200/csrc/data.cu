@@ -46,15 +46,6 @@ void launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem
   cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);  // errors: cudaGetLastError
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat16 l = __float2bfloat16_rn(lo);
-  const __nv_bfloat16 h = __float2bfloat16_rn(hi);
-  return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
-}
-
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));

@@ -2,6 +2,7 @@
 // workspace layout, config validation, device helpers.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -169,6 +170,15 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 // home rank of expert e (e / L) without a division
 __device__ __forceinline__ int home_of(const Dims &d, int e) {
   return d.L == 1 ? e : (int)__umulhi((unsigned)e, d.magicL);
+}
+
+// bf16 pairs packed in a 32-bit word: exact widening, and round-to-nearest-even packing
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat16 l = __float2bfloat16_rn(lo);
+  const __nv_bfloat16 h = __float2bfloat16_rn(hi);
+  return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -1416,7 +1416,107 @@ __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
   }
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+// Data phases of the fused forward layer (plan_fused_kernel): the buffers of the
+// identity-expert layer and the dispatch chunking of a token row.
+struct FusedArgs {
+  const float *gates;  // [N]
+  const uint4 *x;      // [R*S, H/8]
+  uint4 *recv;         // [R*NvS, H/8]
+  uint4 *out;          // [R*S, H/8]
+  int64_t nvec;        // H / 8
+  int64_t nch;         // column chunks a token row is cut into for dispatch
+  int64_t cl;          // vectors per chunk (<= 32 * kFusedU)
+};
+constexpr int kFusedU = 14;  // dispatch: 16-byte vectors per lane of a column chunk
+
+// Zero-copy dispatch of this CTA's tokens [t0, t1): a warp loads a column chunk of a
+// token row once (kFusedU vectors per lane in flight) and stores it to the token's K
+// rows (srow: the rows of the chunk's pairs, pair order).
+__device__ void fused_dispatch(const FusedArgs &f, int64_t t0, int64_t t1, int K, const int *srow) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nunits = (t1 - t0) * f.nch;
+  for (int64_t u = warp; u < nunits; u += kPlanWarps) {
+    const int64_t tl = u / f.nch, t = t0 + tl;
+    const int64_t c0 = (u - tl * f.nch) * f.cl;
+    const int64_t c1 = c0 + f.cl < f.nvec ? c0 + f.cl : f.nvec;
+    const uint4 *src = f.x + t * f.nvec;
+    uint4 buf[kFusedU];
+#pragma unroll
+    for (int q = 0; q < kFusedU; q++) {
+      const int64_t v = c0 + q * 32 + lane;
+      if (v < c1) buf[q] = __ldcs(src + v);
+    }
+    for (int k = 0; k < K; k++) {
+      const int row = srow[tl * K + k];
+      if (row < 0) continue;
+      uint4 *dst = f.recv + (int64_t)row * f.nvec;
+#pragma unroll
+      for (int q = 0; q < kFusedU; q++) {
+        const int64_t v = c0 + q * 32 + lane;
+        if (v < c1) dst[v] = buf[q];
+      }
+    }
+  }
+}
+
+// Combine of this CTA's tokens from the rows it has just dispatched (identity expert:
+// y = recv): a warp per token, the K rows of a column chunk loaded before any
+// arithmetic, fused multiply-adds in ascending k, one rounding to bf16.
+__device__ void fused_combine(const FusedArgs &f, int64_t t0, int64_t t1, int K, const int *srow) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t t = t0 + warp; t < t1; t += kPlanWarps) {
+    const int my_slot = lane < K ? srow[(t - t0) * K + lane] : -1;
+    const float my_w = lane < K ? __ldg(f.gates + t * K + lane) : 0.f;
+    int rows[8];
+    float ws[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      rows[k] = __shfl_sync(0xffffffffu, my_slot, k);
+      ws[k] = __shfl_sync(0xffffffffu, my_w, k);
+    }
+    for (int64_t v0 = 0; v0 < f.nvec; v0 += 64) {
+      uint4 q[8][2];
+#pragma unroll
+      for (int k = 0; k < 8; k++)
+#pragma unroll
+        for (int uu = 0; uu < 2; uu++) {
+          const int64_t v = v0 + uu * 32 + lane;
+          q[k][uu] = (rows[k] >= 0 && v < f.nvec) ? __ldcg(f.recv + (int64_t)rows[k] * f.nvec + v)
+                                                  : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+      for (int uu = 0; uu < 2; uu++) {
+        const int64_t v = v0 + uu * 32 + lane;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          if (rows[k] < 0) continue;  // k >= K, or a pair without a slot
+          const uint32_t wd[4] = {q[k][uu].x, q[k][uu].y, q[k][uu].z, q[k][uu].w};
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            acc[2 * i] = __fmaf_rn(ws[k], bf16_lo(wd[i]), acc[2 * i]);
+            acc[2 * i + 1] = __fmaf_rn(ws[k], bf16_hi(wd[i]), acc[2 * i + 1]);
+          }
+        }
+        if (v < f.nvec) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[0], acc[1]);
+          o.y = pack_bf16x2(acc[2], acc[3]);
+          o.z = pack_bf16x2(acc[4], acc[5]);
+          o.w = pack_bf16x2(acc[6], acc[7]);
+          f.out[t * f.nvec + v] = o;
+        }
+      }
+    }
+  }
+}
+
+// kFused: the plan followed, in the same launch, by the dispatch of this CTA's tokens
+// and the combine of the same tokens (identity expert; a chunk holds whole tokens).
+template <bool kFused>
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArgs f) {
   // launched with programmatic stream serialisation: wait here until the kernel
   // before it in the stream (the router's top-k, the previous layer) has completed
   // and its writes are visible
@@ -1468,6 +1568,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
         sc[S_BAD] = st;
       }
     }
+    if (kFused) {  // as the separate calls would: nothing dispatched, every output row zero
+      const int64_t t0 = k * a.ch / d.K;
+      const int64_t t1 = ((k + 1) * a.ch < d.N ? (k + 1) * a.ch : d.N) / d.K;
+      for (int64_t q = t0 * f.nvec + tid; q < t1 * f.nvec; q += kPlanThreads) f.out[q] = make_uint4(0, 0, 0, 0);
+    }
     return;
   }
   // place this chunk's pairs
@@ -1485,10 +1590,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       if (row < 0 || row >= nrows) row = -1;  // unreachable for a consistent plan
       slot_of[p] = row;
       if (row >= 0) slot_src[row] = (int32_t)p;
+      if (kFused) m.tmp[p - k * a.ch] = row;  // the chunk's rows, pair order
     }
+  }
+  if (kFused) {
+    // a chunk holds whole tokens (K divides 512): every row a token's combine reads was
+    // written by this CTA's dispatch, so a CTA barrier orders the two phases
+    const int K = (int)d.K;
+    const int64_t t0 = k * a.ch / K;
+    const int64_t t1 = ((k + 1) * a.ch < d.N ? (k + 1) * a.ch : d.N) / K;
+    __syncthreads();
+    fused_dispatch(f, t0, t1, K, m.tmp);
+    __syncthreads();
+    fused_combine(f, t0, t1, K, m.tmp);
   }
   fast_tables(a, m);
 }
+
 
 size_t plan_multichunk_smem_bytes(const Dims &d) {
   const size_t worker = std::max<size_t>(size_t(kPlanWarps) * d.E,
@@ -1513,7 +1631,7 @@ struct KernelLaunchInfo {
 struct DeviceLaunchInfo {
   unsigned long long ctx = 0;
   int sms = 0;
-  KernelLaunchInfo k[2];  // 0: plan_kernel, 1: plan_multichunk_kernel
+  KernelLaunchInfo k[3];  // 0: plan_kernel<false>, 1: plan_multichunk_kernel, 2: plan_kernel<true>
 };
 std::mutex g_launch_mu;
 DeviceLaunchInfo g_launch[kMaxDevices];
@@ -1629,14 +1747,14 @@ extern "C" moonep_status_t moonep_plan_view(const moonep_config_t *cfg, const vo
   return MOONEP_OK;
 }
 
-extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t *topk_idx,
-                                       void *plan_arena, void *workspace, int32_t *dev_status,
-                                       moonep_stream_t stream) {
-  Dims d;
-  if (!make_dims(cfg, &d)) return MOONEP_ERR_INVALID_ARG;
-  if (!plan_arena || !workspace || !dev_status || (d.N > 0 && !topk_idx))
-    return MOONEP_ERR_INVALID_ARG;
-  if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
+namespace moonep {
+namespace {
+// The plan launch shared by moonep_plan and moonep_fused_forward (fused != nullptr: the
+// one-chunk-per-CTA kernel with the data phases, or MOONEP_ERR_UNSUPPORTED when the
+// chunks do not fit on the co-resident CTAs).  Arguments were checked by the caller.
+moonep_status_t launch_plan(const Dims &d, const int32_t *topk_idx, void *plan_arena,
+                            void *workspace, int32_t *dev_status, moonep_stream_t stream,
+                            const FusedArgs *fused) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOONEP_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOONEP_ERR_UNSUPPORTED;
@@ -1646,12 +1764,12 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   // CTAs run at the same time)
   int sms = 0;
   const size_t smem = plan_smem_bytes(d);
-  const int per_sm = plan_ctas_per_sm(plan_kernel, 0, dev, smem, &sms);
+  const int per_sm = fused ? plan_ctas_per_sm(plan_kernel<true>, 2, dev, smem, &sms)
+                           : plan_ctas_per_sm(plan_kernel<false>, 0, dev, smem, &sms);
   if (per_sm < 0) return MOONEP_ERR_CUDA;
   PlanArgs a;
   a.d = d;
   bool one_chunk_per_cta = false;
-  void (*kernel)(PlanArgs) = plan_kernel;
   size_t kernel_smem = smem;
   if (per_sm > 0) {
     const int64_t coresident = (int64_t)sms * per_sm;
@@ -1666,9 +1784,9 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
     }
   }
   if (!one_chunk_per_cta) {
+    if (fused) return MOONEP_ERR_UNSUPPORTED;
     // chunks outnumber the co-resident CTAs: one solving CTA, workers with
     // several chunks each
-    kernel = plan_multichunk_kernel;
     kernel_smem = plan_multichunk_smem_bytes(d);
     const int ms = plan_ctas_per_sm(plan_multichunk_kernel, 1, dev, kernel_smem, &sms);
     if (ms < 0) return MOONEP_ERR_CUDA;
@@ -1700,6 +1818,7 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   a.status = dev_status;
   a.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   a.phantom = g_phantom_arrivals.load(std::memory_order_relaxed);
+  const FusedArgs f = fused ? *fused : FusedArgs{};
 
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3((unsigned)(one_chunk_per_cta ? a.nc : a.workers + 1));
@@ -1712,18 +1831,60 @@ extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = attr;
+  auto go = [&]() {
+    if (!one_chunk_per_cta) return cudaLaunchKernelEx(&lc, plan_multichunk_kernel, a);
+    return fused ? cudaLaunchKernelEx(&lc, plan_kernel<true>, a, f)
+                 : cudaLaunchKernelEx(&lc, plan_kernel<false>, a, f);
+  };
   // programmatic dependent launch hides the launch gap after the previous
   // kernel; without it (a runtime that refuses the pair) the launch is plain
   lc.numAttrs = g_plan_pdl.load(std::memory_order_relaxed) ? 2 : 1;
-  if (cudaLaunchKernelEx(&lc, kernel, a) == cudaSuccess) return MOONEP_OK;
+  if (go() == cudaSuccess) return MOONEP_OK;
   cudaGetLastError();
   if (lc.numAttrs == 2) {
     g_plan_pdl.store(false);
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, kernel, a) == cudaSuccess) return MOONEP_OK;
+    if (go() == cudaSuccess) return MOONEP_OK;
     cudaGetLastError();
   }
   return MOONEP_ERR_CUDA;
+}
+}  // namespace
+}  // namespace moonep
+
+extern "C" moonep_status_t moonep_plan(const moonep_config_t *cfg, const int32_t *topk_idx,
+                                       void *plan_arena, void *workspace, int32_t *dev_status,
+                                       moonep_stream_t stream) {
+  Dims d;
+  if (!make_dims(cfg, &d)) return MOONEP_ERR_INVALID_ARG;
+  if (!plan_arena || !workspace || !dev_status || (d.N > 0 && !topk_idx))
+    return MOONEP_ERR_INVALID_ARG;
+  if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
+  return launch_plan(d, topk_idx, plan_arena, workspace, dev_status, stream, nullptr);
+}
+
+extern "C" moonep_status_t moonep_fused_forward(const moonep_config_t *cfg, const int32_t *topk_idx,
+                                                const float *gates, const uint16_t *x,
+                                                void *plan_arena, void *workspace, uint16_t *recv,
+                                                uint16_t *out, int32_t *dev_status,
+                                                moonep_stream_t stream) {
+  Dims d;
+  if (!make_dims(cfg, &d) || d.H < 1) return MOONEP_ERR_INVALID_ARG;
+  if (!plan_arena || !workspace || !dev_status) return MOONEP_ERR_INVALID_ARG;
+  if (d.N > 0 && (!topk_idx || !gates || !x || !recv || !out)) return MOONEP_ERR_INVALID_ARG;
+  if (!aligned256(plan_arena) || !aligned256(workspace)) return MOONEP_ERR_INVALID_ARG;
+  // whole tokens per chunk (chunks are multiples of 512 pairs), 16-byte rows, K <= 8
+  if (kPlanThreads % d.K != 0 || d.K > 8 || d.H % 8 != 0) return MOONEP_ERR_UNSUPPORTED;
+  if (d.N > 0 && (!aligned16(x) || !aligned16(recv) || !aligned16(out))) return MOONEP_ERR_UNSUPPORTED;
+  FusedArgs f;
+  f.gates = gates;
+  f.x = reinterpret_cast<const uint4 *>(x);
+  f.recv = reinterpret_cast<uint4 *>(recv);
+  f.out = reinterpret_cast<uint4 *>(out);
+  f.nvec = d.H / 8;
+  f.nch = (f.nvec + 32 * kFusedU - 1) / (32 * kFusedU);
+  f.cl = (f.nvec + f.nch - 1) / f.nch;
+  return launch_plan(d, topk_idx, plan_arena, workspace, dev_status, stream, &f);
 }
 
 namespace moonep {
