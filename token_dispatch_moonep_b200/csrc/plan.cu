@@ -47,6 +47,8 @@ constexpr int kStBad = 1, kStCapacity = 2, kStTimeout = 8;
 // epochs, constant fills, zeros) never equal the next epoch by accident.
 constexpr unsigned kEpochStep = 0x9E3779B1u;
 constexpr int kSyncGen = 0, kSyncDone = 1, kSyncState = 2, kSyncTables = 3;
+// tags of the two expert-total buffers: the epoch of the launch each was zeroed for
+constexpr int kSyncTotTag = 4;
 
 struct PlanArgs {
   Dims d;
@@ -56,7 +58,8 @@ struct PlanArgs {
   int64_t nc;     // chunks
   const int32_t *idx;
   PlanPtrs P;
-  int32_t *sync;     // generation, done, state, tables-done
+  int32_t *sync;     // generation, done, state, tables-done, totals tags
+  int32_t *totals;   // [2][MOONEP_MAX_EXPERTS] expert totals, one buffer per epoch parity
   int32_t *arrive;   // [nc + phantom] per-chunk arrival epochs
   int32_t *badmark;  // [nc]
   int32_t *hist;     // [nc][E] chunk histograms (rewritten as bases when chunks > workers)
@@ -217,9 +220,11 @@ __device__ void column_sums(const int32_t *hist, int E, int64_t nrows, int *out,
 // chunk's pairs of the same expert.  Pair of (warp w, step j, lane l) is
 // k*ch + w*32*ppt + j*32 + l.  ev[j]: expert id, -1 bad id, -2 past the end.
 // kU16: the histogram row is written as uint16 (a chunk holds at most 8192 pairs).
+// chunk_tot (may be null): the chunk's count of each expert, in shared memory.
 template <bool kU16>
 __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *wh,
-                                            int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread]) {
+                                            int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread],
+                                            int *chunk_tot = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = (int)a.d.E, ppt = a.ppt;
   for (int i = tid; i < kPlanWarps * E; i += kPlanThreads) wh[i] = 0;
@@ -266,6 +271,7 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
       reinterpret_cast<uint16_t *>(a.hist)[k * E + e] = (uint16_t)acc;
     else
       a.hist[k * E + e] = acc;
+    if (chunk_tot) chunk_tot[e] = acc;
   }
   __syncthreads();
 #pragma unroll
@@ -1050,6 +1056,85 @@ __device__ int gather_all(const PlanArgs &a, int64_t k, int epoch, const FastSme
   return m.misc[M_STATE];
 }
 
+// Barrier of the first NT threads of the block: __syncthreads for the whole block,
+// else named barrier BAR (the other threads of the block do other work meanwhile).
+template <int NT, int BAR>
+__device__ __forceinline__ void group_sync() {
+  if (NT == kPlanThreads) __syncthreads();
+  else asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
+// Warps 8..15 of the split gather: m.base[e] = pairs of expert e in the chunks before
+// chunk k, read from the nearer end: the rows before k when k < nc / 2, else the
+// totals less the rows from k on (no CTA reads more than half the rows).  A row is
+// U = E / V units of V counts; G groups of the 256 threads take rows r, r + G, ...
+template <int V>
+__device__ void chunk_bases_split(const PlanArgs &a, int64_t k, const int32_t *totals,
+                                  const FastSmem &m) {
+  constexpr int NT = kPlanThreads / 2;
+  const int tb = threadIdx.x - NT;
+  const int E = (int)a.d.E;
+  const uint16_t *hist = reinterpret_cast<const uint16_t *>(a.hist);
+  const bool suffix = 2 * k >= a.nc;
+  const int64_t r_lo = suffix ? k : 0, r_hi = suffix ? a.nc : k;
+  const int U = E / V;
+  const int gw = U < NT ? U : NT;
+  const int G = NT / gw;
+  const int g = tb / gw, u0 = tb % gw;
+  const int NU = (U + gw - 1) / gw;
+  constexpr int QN = V == 8 ? 1 : 4;  // E <= 1024: U <= 128 units of 8, or <= 1024 of 1
+  int acc[QN][V];
+#pragma unroll
+  for (int q = 0; q < QN; q++)
+#pragma unroll
+    for (int v = 0; v < V; v++) acc[q][v] = 0;
+  if (g < G) {
+    for (int64_t r0 = r_lo + g; r0 < r_hi; r0 += 8LL * G) {
+      uint32_t vals[8][QN][V == 8 ? 4 : 1];
+#pragma unroll
+      for (int j = 0; j < 8; j++) {  // the batch's loads first, then the sums
+        const int64_t r = r0 + (int64_t)j * G;
+#pragma unroll
+        for (int q = 0; q < QN; q++) {
+          const int u = u0 + q * gw;
+          const bool in = r < r_hi && q < NU && u < U;
+          if constexpr (V == 8) {
+            const uint4 t = in ? __ldcg(reinterpret_cast<const uint4 *>(hist + r * E) + u)
+                               : make_uint4(0, 0, 0, 0);
+            vals[j][q][0] = t.x;
+            vals[j][q][1] = t.y;
+            vals[j][q][2] = t.z;
+            vals[j][q][3] = t.w;
+          } else {
+            vals[j][q][0] = in ? __ldcg(hist + r * E + u) : 0u;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j++)
+#pragma unroll
+        for (int q = 0; q < QN; q++)
+#pragma unroll
+          for (int v = 0; v < V; v++)
+            acc[q][v] += V == 8 ? (int)((vals[j][q][v >> 1] >> ((v & 1) * 16)) & 0xffffu)
+                                : (int)vals[j][q][0];
+    }
+#pragma unroll
+    for (int q = 0; q < QN; q++) {
+      const int u = u0 + q * gw;
+      if (q >= NU || u >= U) break;
+#pragma unroll
+      for (int v = 0; v < V; v++) m.tmp[g * E + u * V + v] = acc[q][v];
+    }
+  }
+  group_sync<NT, 2>();
+  for (int e = tb; e < E; e += NT) {
+    int sum = 0;
+    for (int q = 0; q < G; q++) sum += m.tmp[q * E + e];
+    m.base[e] = suffix ? __ldcg(totals + e) - sum : sum;
+  }
+}
+
 // first i in [0, n) with a[i] > v (n if none); a non-decreasing.  The steps depend only
 // on n (no data-dependent branches): the same trip count for every thread.
 __device__ __forceinline__ int upper_bound_bf(const int *a, int n, int v) {
@@ -1064,10 +1149,10 @@ __device__ __forceinline__ int upper_bound_bf(const int *a, int n, int v) {
   return (int)(base - a) + (*base <= v ? 1 : 0);
 }
 
-// Exclusive scan over the block of NA values per thread, in thread order, with the
-// totals: one barrier.  Each call passes its own scratch area (NA * kPlanWarps ints) so
-// that no second barrier is needed before the area is written again.
-template <int NA>
+// Exclusive scan over the NT threads of NA values per thread, in thread order, with
+// the totals: one barrier.  Each call passes its own scratch area (NA * kPlanWarps
+// ints) so that no second barrier is needed before the area is written again.
+template <int NA, int NT, int BAR>
 __device__ __forceinline__ void block_scan(const int (&v)[NA], int (&ex)[NA], int (&tot)[NA],
                                            int *scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1077,12 +1162,12 @@ __device__ __forceinline__ void block_scan(const int (&v)[NA], int (&ex)[NA], in
   if (lane == 31)
 #pragma unroll
     for (int k = 0; k < NA; k++) scratch[k * kPlanWarps + warp] = inc[k];
-  __syncthreads();
+  group_sync<NT, BAR>();
 #pragma unroll
   for (int k = 0; k < NA; k++) {
     int off = 0, t = 0;
 #pragma unroll
-    for (int w = 0; w < kPlanWarps; w++) {
+    for (int w = 0; w < NT / 32; w++) {
       const int x = scratch[k * kPlanWarps + w];
       off += w < warp ? x : 0;
       t += x;
@@ -1092,30 +1177,32 @@ __device__ __forceinline__ void block_scan(const int (&v)[NA], int (&ex)[NA], in
   }
 }
 
-// Thread t's contiguous share [b, e) of n elements (n <= 4 * kPlanThreads).
+// Thread t's contiguous share [b, e) of n elements among NT threads.
+template <int NT>
 __device__ __forceinline__ void share_of(int n, int &b, int &e) {
-  const int per = (n + kPlanThreads - 1) / kPlanThreads;
+  const int per = (n + NT - 1) / NT;
   b = min((int)threadIdx.x * per, n);
   e = min(b + per, n);
 }
 
-// The balance problem, from m.cnt, by the whole block (the fixed rule of the plan; see
-// the file header): block scans over experts, ranks and pieces, one thread per element
-// in between.  Writes the solve state into shared memory; misc[M_CAP] != 0 if a rank
+// The balance problem, from m.cnt, by the first NT threads of the block (the fixed
+// rule of the plan; see the file header): block scans over experts, ranks and pieces,
+// one thread per element in between.  Writes the solve state into shared memory; misc[M_CAP] != 0 if a rank
 // would pass NvS rows or the tables do not fit together (unreachable).
+template <int NT, int BAR>
 __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   const int tid = threadIdx.x;
   const int E = (int)d.E, R = (int)d.R, L = (int)d.L, A = (int)d.A, B = (int)d.B;
   const int SK = (int)d.SK, NvS = (int)d.NvS, N = (int)d.N, PM = (int)d.PMAX;
   int *scr = m.scratch;  // 8 areas of 4 * kPlanWarps ints
   int eb, ee, hb, he;
-  share_of(E, eb, ee);
-  share_of(R, hb, he);
+  share_of<NT>(E, eb, ee);
+  share_of<NT>(R, hb, he);
   // (1) global exclusive prefix of the expert counts
   {
     int v[1] = {0}, ex[1], tot[1];
     for (int e = eb; e < ee; e++) v[0] += m.cnt[e];
-    block_scan<1>(v, ex, tot, scr);
+    block_scan<1, NT, BAR>(v, ex, tot, scr);
     int run = ex[0];
     for (int e = eb; e < ee; e++) {
       m.gcst[e] = run;
@@ -1126,7 +1213,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       m.misc[M_NREMOTE] = 0;
     }
   }
-  __syncthreads();
+  group_sync<NT, BAR>();
   // (2) rank loads; overflow and deficit bases; the receivers (ranks below S*K) in rank order
   int n_recv;
   {
@@ -1138,7 +1225,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       v[1] += ld < SK ? SK - ld : 0;
       v[2] += ld < SK ? 1 : 0;
     }
-    block_scan<3>(v, ex, tot, scr + 4 * kPlanWarps);
+    block_scan<3, NT, BAR>(v, ex, tot, scr + 4 * kPlanWarps);
     int ov = ex[0], df = ex[1], rf = ex[2];
     for (int h = hb; h < he; h++) {
       const int ld = m.load[h];
@@ -1160,7 +1247,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     }
     n_recv = tot[2];
   }
-  __syncthreads();
+  group_sync<NT, BAR>();
   // (3) per expert: rows kept at home, its range [oend - ovf, oend) of the overflow
   //     stream, the receivers it reaches (one piece each); piece ids and padded kept rows
   //     by one scan
@@ -1191,7 +1278,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       v[0] += npc;
       v[1] += A > 1 ? roundup_i(kept, A) : kept;
     }
-    block_scan<2>(v, ex, tot, scr + 8 * kPlanWarps);
+    block_scan<2, NT, BAR>(v, ex, tot, scr + 8 * kPlanWarps);
     int rp = ex[0], rk = ex[1];
     for (int e = eb; e < ee; e++) {
       m.pid0[e] = rp;
@@ -1203,11 +1290,11 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     n_piece = tot[0] < PM ? tot[0] : PM;  // pieces <= experts + receivers - 1 < PMAX
     padtot = tot[1];
   }
-  __syncthreads();
+  group_sync<NT, BAR>();
   // (4) one task per thread: an expert's segment start and first row; a rank's native
   //     rows; a piece's expert, receiver and range; a receiver's first piece and count
   int bad = 0;
-  for (int t = tid; t < E + R + n_piece + n_recv; t += kPlanThreads) {
+  for (int t = tid; t < E + R + n_piece + n_recv; t += NT) {
     if (t < E) {
       const int e = t, h = home_of(d, e);
       const int nst = m.epos[e] - m.epos[h * L];
@@ -1248,29 +1335,29 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     }
   }
   if (bad) atomicOr(&m.misc[M_CAP], 1);
-  __syncthreads();
+  group_sync<NT, BAR>();
   // (5) alignment > 1: a piece's start is its receiver's native rows plus the padded
   //     lengths of the receiver's earlier pieces (a scan over the pieces)
   if (A > 1) {
     int pb, pe;
-    share_of(n_piece, pb, pe);
+    share_of<NT>(n_piece, pb, pe);
     int v[1] = {0}, ex[1], tot[1];
     for (int pid = pb; pid < pe; pid++) v[0] += m.pscan[pid];
-    block_scan<1>(v, ex, tot, scr + 16 * kPlanWarps);
-    __syncthreads();  // every thread has read its values before they are overwritten
+    block_scan<1, NT, BAR>(v, ex, tot, scr + 16 * kPlanWarps);
+    group_sync<NT, BAR>();  // every thread has read its values before they are overwritten
     int run = ex[0];
     for (int pid = pb; pid < pe; pid++) {
       const int x = m.pscan[pid];
       m.pscan[pid] = run;
       run += x;
     }
-    __syncthreads();
+    group_sync<NT, BAR>();
   }
   // (6) one piece per thread: its first row within the receiving rank (alignment 1: the
   //     receiver's rows follow its native rows in overflow-stream order), capacity,
   //     local-replica flags, remote pieces
   int cap = 0, nrem = 0;
-  for (int pid = tid; pid < n_piece; pid += kPlanThreads) {
+  for (int pid = tid; pid < n_piece; pid += NT) {
     const int i = m.precv[pid], first = m.rfirst[i], dr = m.rrank[i];
     if (pid < first) cap = 1;
     const int st = A > 1 ? m.ntot[dr] + m.pscan[pid] - m.pscan[first]
@@ -1281,7 +1368,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     if (pid - first < B) m.eflag[m.pexp[pid]] = 1;
     else nrem++;
   }
-  for (int h = tid; h < R; h += kPlanThreads)
+  for (int h = tid; h < R; h += NT)
     if (m.ntot[h] > NvS) cap = 1;
   if (cap) atomicOr(&m.misc[M_CAP], 1);
   if (nrem) atomicAdd(&m.misc[M_NREMOTE], nrem);
@@ -1289,7 +1376,37 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     m.misc[M_NRECV] = n_recv;
     m.misc[M_NPIECE] = n_piece;
   }
+  group_sync<NT, BAR>();
+}
+
+// The gather when this launch's expert totals were added up by atomics (every chunk
+// adds its counts before it arrives): warp 0 waits for the arrivals; then warps 0..7
+// read the totals and solve while warps 8..15 work out the chunk's base offsets.
+// Returns the state bits (kStTimeout, kStBad); the solve is done when it returns 0.
+template <int V>
+__device__ int gather_split(const PlanArgs &a, int64_t k, int epoch, const int32_t *totals,
+                            const FastSmem &m) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = (int)a.d.E;
+  if (tid < 32) {
+    const bool ok = warp_wait_all(a.arrive, a.nc + a.phantom, epoch, a.wait_ns);
+    if (lane == 0) m.misc[M_STATE] = ok ? 0 : kStTimeout;
+  }
   __syncthreads();
+  if (m.misc[M_STATE]) return kStTimeout;
+  if (warp < kPlanWarps / 2) {
+    constexpr int NT = kPlanThreads / 2;
+    for (int e = tid; e < E; e += NT) m.cnt[e] = __ldcg(totals + e);
+    bool bad = false;
+    for (int64_t c = tid; c < a.nc; c += NT) bad |= __ldcg(a.badmark + c) == epoch;
+    if (bad) atomicOr(&m.misc[M_STATE], kStBad);
+    group_sync<NT, 1>();
+    if (m.misc[M_STATE] == 0) solve_fast<NT, 1>(a.d, m);
+  } else {
+    chunk_bases_split<V>(a, k, totals, m);
+  }
+  __syncthreads();
+  return m.misc[M_STATE];
 }
 
 // Row of a pair at position pos of expert e's list (solve state in shared memory).
@@ -1522,34 +1639,64 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
   // and its writes are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) int smem[];
-  __shared__ int s_epoch;
+  __shared__ int s_epoch, s_fast;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const Dims &d = a.d;
   const int64_t k = blockIdx.x;  // this CTA's chunk
   const FastSmem m = carve_fast(d, smem);
   int32_t *gen = a.sync + kSyncGen;
-  // the generation word: needed only when the chunk is published, so its load
-  // overlaps the counting
-  int gen_v = 0;
-  if (tid == 0) gen_v = *((volatile int32_t *)gen);
+  // the generation word and the two totals tags: needed only when the chunk is
+  // published, so their loads overlap the counting (the previous launch has completed,
+  // so plain loads see its writes)
+  int gen_v = 0, tag0 = 0, tag1 = 0;
+  if (tid == 0) {
+    gen_v = *((volatile int32_t *)gen);
+    tag0 = *((volatile int32_t *)(a.sync + kSyncTotTag));
+    tag1 = *((volatile int32_t *)(a.sync + kSyncTotTag + 1));
+  }
   int ev[kPairsPerThread], rk[kPairsPerThread];
-  const bool bad = __syncthreads_or(count_chunk<true>(a, k, m.tmp, ev, rk));
-  if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
+  const bool bad = __syncthreads_or(count_chunk<true>(a, k, m.tmp, ev, rk, m.base));
+  if (tid == 0) {
+    const int e = (int)((unsigned)gen_v + kEpochStep);
+    s_epoch = e;
+    // the totals buffer of this epoch's parity was zeroed for exactly this epoch by the
+    // launch before (else: first use of the workspace, or it ran another kernel)
+    s_fast = ((e & 1) ? tag1 : tag0) == e;
+  }
   __syncthreads();
   const int epoch = s_epoch;
+  const bool fast = s_fast;
+  int32_t *totals = a.totals + (epoch & 1) * MOONEP_MAX_EXPERTS;
+  if (fast) {
+    for (int e = tid; e < (int)d.E; e += kPlanThreads)
+      if (m.base[e]) atomicAdd(totals + e, m.base[e]);
+    __syncthreads();
+  }
   if (tid == 0) {
     if (bad) set_status(a.status, MOONEP_DEV_BAD_EXPERT_ID);
     a.badmark[k] = bad ? epoch : ~epoch;
-    // the histogram row was written by every thread before the barriers above; the
-    // release store orders all of it (barrier, then release: cumulative) before the flag
+    // the histogram row and the totals were written by every thread before the
+    // barriers above; the release store orders all of it (barrier, then release:
+    // cumulative) before the flag
     st_release(a.arrive + k, epoch);
   }
-  int st = (d.E & 7) == 0 ? gather_all<8>(a, k, epoch, m) : gather_all<1>(a, k, epoch, m);
+  if (k == 0) {  // zero the other buffer for the next launch (nobody uses it in this one)
+    const int nxt = (epoch & 1) ^ 1;
+    int32_t *other = a.totals + nxt * MOONEP_MAX_EXPERTS;
+    for (int e = tid; e < MOONEP_MAX_EXPERTS; e += kPlanThreads) other[e] = 0;
+    __syncthreads();
+    if (tid == 0) st_release(a.sync + kSyncTotTag + nxt, (int)((unsigned)epoch + kEpochStep));
+  }
+  int st;
+  if (fast)
+    st = (d.E & 7) == 0 ? gather_split<8>(a, k, epoch, totals, m) : gather_split<1>(a, k, epoch, totals, m);
+  else
+    st = (d.E & 7) == 0 ? gather_all<8>(a, k, epoch, m) : gather_all<1>(a, k, epoch, m);
   // every CTA has arrived, so every CTA has read the generation word; a bad id
   // does not stop this, the next launch must get a new epoch in any case
   if (k == 0 && tid == 0) *((volatile int32_t *)gen) = epoch;
   if (st == 0) {
-    solve_fast(d, m);
+    if (!fast) solve_fast<kPlanThreads, 0>(d, m);
     if (m.misc[M_CAP]) st = kStCapacity;
   }
   int32_t *slot_of = a.P.f[F_SLOT_OF];
@@ -1807,6 +1954,7 @@ moonep_status_t launch_plan(const Dims &d, const int32_t *topk_idx, void *plan_a
   WsLayout wl(d);
   char *ws = static_cast<char *>(workspace);
   a.sync = reinterpret_cast<int32_t *>(ws + wl.off[W_SYNC]);
+  a.totals = reinterpret_cast<int32_t *>(ws + wl.off[W_TOTALS]);
   a.arrive = reinterpret_cast<int32_t *>(ws + wl.off[W_ARRIVE]);
   a.badmark = reinterpret_cast<int32_t *>(ws + wl.off[W_BADMARK]);
   a.hist = reinterpret_cast<int32_t *>(ws + wl.off[W_HIST]);
