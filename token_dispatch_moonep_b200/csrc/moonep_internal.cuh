@@ -115,12 +115,14 @@ inline PlanPtrs plan_ptrs(const Dims &d, const void *arena) {
 
 // -------------------------------------------------------------- workspace ---
 // Plan scratch: sync words (generation, done, state, tables-done, two totals
-// tags), two expert-total buffers of MOONEP_MAX_EXPERTS counts at a fixed offset
+// tags), two expert-total buffers (each kTotalCopies partial copies of
+// MOONEP_MAX_EXPERTS counts) at a fixed offset
 // (so that a call with another config finds them where the last call left them),
 // per-chunk arrival epochs (plus slots for diagnostic phantom arrivals), per-chunk
 // bad-id marks, per-chunk histograms, stable ranks, placement constants.
 constexpr int kSyncWords = 16;
 constexpr int kSyncMaxPhantom = 32;
+constexpr int kTotalCopies = 16;  // chunk k adds its counts into copy k % 16 (spreads the atomics)
 
 enum WsField {
   W_SYNC, W_TOTALS, W_ARRIVE, W_BADMARK, W_HIST, W_RANK, W_EXP_KEPT, W_EXP_ROW0, W_EXP_OSTART,
@@ -133,7 +135,7 @@ struct WsLayout {
   explicit WsLayout(const Dims &d) {
     const size_t n[W_COUNT] = {
         size_t(kSyncWords) * sizeof(int32_t),
-        size_t(2 * MOONEP_MAX_EXPERTS) * sizeof(int32_t),
+        size_t(2 * kTotalCopies * MOONEP_MAX_EXPERTS) * sizeof(int32_t),
         size_t(d.NCMAX + kSyncMaxPhantom) * sizeof(int32_t),
         size_t(d.NCMAX) * sizeof(int32_t),
         size_t(d.E * d.NCMAX) * sizeof(int32_t),

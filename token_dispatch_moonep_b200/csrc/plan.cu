@@ -59,7 +59,7 @@ struct PlanArgs {
   const int32_t *idx;
   PlanPtrs P;
   int32_t *sync;     // generation, done, state, tables-done, totals tags
-  int32_t *totals;   // [2][MOONEP_MAX_EXPERTS] expert totals, one buffer per epoch parity
+  int32_t *totals;   // [2][kTotalCopies][MOONEP_MAX_EXPERTS] expert totals, a buffer per epoch parity
   int32_t *arrive;   // [nc + phantom] per-chunk arrival epochs
   int32_t *badmark;  // [nc]
   int32_t *hist;     // [nc][E] chunk histograms (rewritten as bases when chunks > workers)
@@ -246,11 +246,19 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
   __syncthreads();
   int *myh = wh + warp * E;
   const uint32_t lt = lanemask_lt();
+  // lanes holding the same id: one ballot per bit of the key id + 2 (id -1: a bad id,
+  // -2: past the end), a fixed cost however many distinct ids the warp holds
+  const int nbits = 32 - __clz(E + 1);
 #pragma unroll
   for (int j = 0; j < kPairsPerThread; j++) {
     if (j >= ppt) break;  // uniform across the block
     const int e = ev[j];
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);  // lanes holding the same id
+    const unsigned key = (unsigned)(e + 2);
+    uint32_t peers = 0xffffffffu;
+    for (int b = 0; b < nbits; b++) {
+      const uint32_t ones = __ballot_sync(0xffffffffu, (key >> b) & 1u);
+      peers &= ((key >> b) & 1u) ? ones : ~ones;
+    }
     const int prev = e >= 0 ? myh[e] : 0;
     const int r = __popc(peers & lt);
     rk[j] = prev + r;
@@ -922,7 +930,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_multichunk_kernel(PlanArgs 
 // One grid-wide exchange (the arrivals) per plan.
 struct FastSmem {
   int *cnt, *base, *gcst, *kept, *ovf, *oend, *nst, *row0, *npc, *i0, *pid0, *eflag, *epos;  // [E]
-  int *load, *over, *def, *ridx, *ntot, *nseg, *rrank, *rbase, *rend, *rfirst, *rstart;  // [R]
+  int *load, *over, *def, *ridx, *ntot, *nseg, *rrank, *rbase, *rend, *rfirst, *rlast;  // [R]
   int *pexp, *precv, *post, *plen, *pst, *prow, *pscan;  // [PMAX]
   int *misc;     // [16]: 0 receivers, 1 pieces, 2 capacity, 3 gather state, 4 remote pieces
   int *scratch;  // 20 * kPlanWarps: the areas of the block scans
@@ -948,7 +956,7 @@ __device__ __forceinline__ FastSmem carve_fast(const Dims &d, int *s) {
                   &m.i0, &m.pid0, &m.eflag, &m.epos};
   for (int i = 0; i < 13; i++) { *ea[i] = s; s += E; }
   int **ra[11] = {&m.load, &m.over, &m.def, &m.ridx, &m.ntot, &m.nseg, &m.rrank, &m.rbase,
-                  &m.rend, &m.rfirst, &m.rstart};
+                  &m.rend, &m.rfirst, &m.rlast};
   for (int i = 0; i < 11; i++) { *ra[i] = s; s += R; }
   int **pa[7] = {&m.pexp, &m.precv, &m.post, &m.plen, &m.pst, &m.prow, &m.pscan};
   for (int i = 0; i < 7; i++) { *pa[i] = s; s += PM; }
@@ -1064,6 +1072,17 @@ __device__ __forceinline__ void group_sync() {
   else asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
 }
 
+// Expert e's total: the sum of its kTotalCopies partial copies (loads in flight together).
+__device__ __forceinline__ int total_of(const int32_t *totals, int e) {
+  int v[kTotalCopies];
+#pragma unroll
+  for (int c = 0; c < kTotalCopies; c++) v[c] = __ldcg(totals + c * MOONEP_MAX_EXPERTS + e);
+  int s = 0;
+#pragma unroll
+  for (int c = 0; c < kTotalCopies; c++) s += v[c];
+  return s;
+}
+
 // Warps 8..15 of the split gather: m.base[e] = pairs of expert e in the chunks before
 // chunk k, read from the nearer end: the rows before k when k < nc / 2, else the
 // totals less the rows from k on (no CTA reads more than half the rows).  A row is
@@ -1131,7 +1150,7 @@ __device__ void chunk_bases_split(const PlanArgs &a, int64_t k, const int32_t *t
   for (int e = tb; e < E; e += NT) {
     int sum = 0;
     for (int q = 0; q < G; q++) sum += m.tmp[q * E + e];
-    m.base[e] = suffix ? __ldcg(totals + e) - sum : sum;
+    m.base[e] = suffix ? total_of(totals, e) - sum : sum;
   }
 }
 
@@ -1193,40 +1212,33 @@ template <int NT, int BAR>
 __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   const int tid = threadIdx.x;
   const int E = (int)d.E, R = (int)d.R, L = (int)d.L, A = (int)d.A, B = (int)d.B;
-  const int SK = (int)d.SK, NvS = (int)d.NvS, N = (int)d.N, PM = (int)d.PMAX;
-  int *scr = m.scratch;  // 8 areas of 4 * kPlanWarps ints
+  const int SK = (int)d.SK, NvS = (int)d.NvS, PM = (int)d.PMAX;
+  int *scr = m.scratch;  // scan areas of 4 * kPlanWarps ints
   int eb, ee, hb, he;
   share_of<NT>(E, eb, ee);
   share_of<NT>(R, hb, he);
-  // (1) global exclusive prefix of the expert counts
+  // (1) one scan for two prefixes: the expert counts (global exclusive prefix) and, over
+  //     the ranks, overflow, deficit and receivers (rank loads are sums of their experts'
+  //     counts); then the receivers (ranks below S*K) in rank order
+  int n_recv;
   {
-    int v[1] = {0}, ex[1], tot[1];
+    int v[4] = {0, 0, 0, 0}, ex[4], tot[4];
     for (int e = eb; e < ee; e++) v[0] += m.cnt[e];
-    block_scan<1, NT, BAR>(v, ex, tot, scr);
+    for (int h = hb; h < he; h++) {
+      int ld = 0;
+      for (int e = h * L; e < (h + 1) * L; e++) ld += m.cnt[e];
+      m.load[h] = ld;
+      v[1] += ld > SK ? ld - SK : 0;
+      v[2] += ld < SK ? SK - ld : 0;
+      v[3] += ld < SK ? 1 : 0;
+    }
+    block_scan<4, NT, BAR>(v, ex, tot, scr);
     int run = ex[0];
     for (int e = eb; e < ee; e++) {
       m.gcst[e] = run;
       run += m.cnt[e];
     }
-    if (tid == 0) {
-      m.misc[M_CAP] = 0;
-      m.misc[M_NREMOTE] = 0;
-    }
-  }
-  group_sync<NT, BAR>();
-  // (2) rank loads; overflow and deficit bases; the receivers (ranks below S*K) in rank order
-  int n_recv;
-  {
-    int v[3] = {0, 0, 0}, ex[3], tot[3];
-    for (int h = hb; h < he; h++) {
-      const int ld = ((h + 1) * L < E ? m.gcst[(h + 1) * L] : N) - m.gcst[h * L];
-      m.load[h] = ld;
-      v[0] += ld > SK ? ld - SK : 0;
-      v[1] += ld < SK ? SK - ld : 0;
-      v[2] += ld < SK ? 1 : 0;
-    }
-    block_scan<3, NT, BAR>(v, ex, tot, scr + 4 * kPlanWarps);
-    int ov = ex[0], df = ex[1], rf = ex[2];
+    int ov = ex[1], df = ex[2], rf = ex[3];
     for (int h = hb; h < he; h++) {
       const int ld = m.load[h];
       const int o = ld > SK ? ld - SK : 0, dd = ld < SK ? SK - ld : 0;
@@ -1245,10 +1257,14 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       ov += o;
       df += dd;
     }
-    n_recv = tot[2];
+    n_recv = tot[3];
+    if (tid == 0) {
+      m.misc[M_CAP] = 0;
+      m.misc[M_NREMOTE] = 0;
+    }
   }
   group_sync<NT, BAR>();
-  // (3) per expert: rows kept at home, its range [oend - ovf, oend) of the overflow
+  // (2) per expert: rows kept at home, its range [oend - ovf, oend) of the overflow
   //     stream, the receivers it reaches (one piece each); piece ids and padded kept rows
   //     by one scan
   int n_piece, padtot;
@@ -1278,7 +1294,8 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       v[0] += npc;
       v[1] += A > 1 ? roundup_i(kept, A) : kept;
     }
-    block_scan<2, NT, BAR>(v, ex, tot, scr + 8 * kPlanWarps);
+    for (int i = tid; i < n_recv; i += NT) m.rfirst[i] = m.rlast[i] = -1;  // set by its pieces
+    block_scan<2, NT, BAR>(v, ex, tot, scr + 4 * kPlanWarps);
     int rp = ex[0], rk = ex[1];
     for (int e = eb; e < ee; e++) {
       m.pid0[e] = rp;
@@ -1291,10 +1308,11 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     padtot = tot[1];
   }
   group_sync<NT, BAR>();
-  // (4) one task per thread: an expert's segment start and first row; a rank's native
-  //     rows; a piece's expert, receiver and range; a receiver's first piece and count
+  // (3) one task per thread: an expert's segment start and first row; a rank's native
+  //     rows; a piece's expert, receiver and range (a piece that starts at its
+  //     receiver's base is the receiver's first, one that ends at its end the last)
   int bad = 0;
-  for (int t = tid; t < E + R + n_piece + n_recv; t += NT) {
+  for (int t = tid; t < E + R + n_piece; t += NT) {
     if (t < E) {
       const int e = t, h = home_of(d, e);
       const int nst = m.epos[e] - m.epos[h * L];
@@ -1303,10 +1321,10 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     } else if (t < E + R) {
       const int h = t - E;
       m.ntot[h] = ((h + 1) * L < E ? m.epos[(h + 1) * L] : padtot) - m.epos[h * L];
-    } else if (t < E + R + n_piece) {
+    } else {
       const int pid = t - E - R;
       const int e = upper_bound_bf(m.pid0, E, pid) - 1;  // its expert: the last first-id <= pid
-      int i = m.i0[e] + (pid - m.pid0[e]);
+      int i = e < 0 ? -1 : m.i0[e] + (pid - m.pid0[e]);
       if (e < 0 || i < 0 || i >= n_recv || pid - m.pid0[e] >= m.npc[e]) {
         bad = 1;
         i = 0;
@@ -1320,30 +1338,20 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       m.post[pid] = os;
       m.plen[pid] = oe - os;
       m.pscan[pid] = A > 1 ? roundup_i(oe - os, A) : oe - os;
-    } else {
-      const int i = t - E - R - n_piece;
-      const int ef = upper_bound_bf(m.oend, E, m.rbase[i]);
-      const int el = upper_bound_bf(m.oend, E, m.rend[i] - 1);
-      int first = ef < E ? m.pid0[ef] + (i - m.i0[ef]) : 0;
-      const int last = el < E ? m.pid0[el] + (i - m.i0[el]) : -1;
-      if (first < 0 || first > last || last >= n_piece || L + (last - first + 1) > E) {
-        bad = 1;
-        first = 0;
-      }
-      m.rfirst[i] = first;
-      m.nseg[m.rrank[i]] = L + (last - first + 1);
+      if (os == m.rbase[i]) m.rfirst[i] = pid;
+      if (oe == m.rend[i]) m.rlast[i] = pid;
     }
   }
   if (bad) atomicOr(&m.misc[M_CAP], 1);
   group_sync<NT, BAR>();
-  // (5) alignment > 1: a piece's start is its receiver's native rows plus the padded
+  // (4) alignment > 1: a piece's start is its receiver's native rows plus the padded
   //     lengths of the receiver's earlier pieces (a scan over the pieces)
   if (A > 1) {
     int pb, pe;
     share_of<NT>(n_piece, pb, pe);
     int v[1] = {0}, ex[1], tot[1];
     for (int pid = pb; pid < pe; pid++) v[0] += m.pscan[pid];
-    block_scan<1, NT, BAR>(v, ex, tot, scr + 16 * kPlanWarps);
+    block_scan<1, NT, BAR>(v, ex, tot, scr + 8 * kPlanWarps);
     group_sync<NT, BAR>();  // every thread has read its values before they are overwritten
     int run = ex[0];
     for (int pid = pb; pid < pe; pid++) {
@@ -1353,13 +1361,16 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     }
     group_sync<NT, BAR>();
   }
-  // (6) one piece per thread: its first row within the receiving rank (alignment 1: the
+  // (5) one piece per thread: its first row within the receiving rank (alignment 1: the
   //     receiver's rows follow its native rows in overflow-stream order), capacity,
-  //     local-replica flags, remote pieces
+  //     local-replica flags, remote pieces; one receiver per thread: its segment count
   int cap = 0, nrem = 0;
   for (int pid = tid; pid < n_piece; pid += NT) {
     const int i = m.precv[pid], first = m.rfirst[i], dr = m.rrank[i];
-    if (pid < first) cap = 1;
+    if (first < 0 || pid < first) {
+      cap = 1;
+      continue;
+    }
     const int st = A > 1 ? m.ntot[dr] + m.pscan[pid] - m.pscan[first]
                          : m.ntot[dr] + (m.post[pid] - m.rbase[i]);
     m.pst[pid] = st;
@@ -1367,6 +1378,11 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     if (st + m.plen[pid] > NvS) cap = 1;
     if (pid - first < B) m.eflag[m.pexp[pid]] = 1;
     else nrem++;
+  }
+  for (int i = tid; i < n_recv; i += NT) {
+    const int first = m.rfirst[i], last = m.rlast[i];
+    if (first < 0 || last < first || L + (last - first + 1) > E) cap = 1;
+    else m.nseg[m.rrank[i]] = L + (last - first + 1);
   }
   for (int h = tid; h < R; h += NT)
     if (m.ntot[h] > NvS) cap = 1;
@@ -1396,7 +1412,7 @@ __device__ int gather_split(const PlanArgs &a, int64_t k, int epoch, const int32
   if (m.misc[M_STATE]) return kStTimeout;
   if (warp < kPlanWarps / 2) {
     constexpr int NT = kPlanThreads / 2;
-    for (int e = tid; e < E; e += NT) m.cnt[e] = __ldcg(totals + e);
+    for (int e = tid; e < E; e += NT) m.cnt[e] = total_of(totals, e);
     bool bad = false;
     for (int64_t c = tid; c < a.nc; c += NT) bad |= __ldcg(a.badmark + c) == epoch;
     if (bad) atomicOr(&m.misc[M_STATE], kStBad);
@@ -1666,10 +1682,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
   __syncthreads();
   const int epoch = s_epoch;
   const bool fast = s_fast;
-  int32_t *totals = a.totals + (epoch & 1) * MOONEP_MAX_EXPERTS;
+  int32_t *totals = a.totals + (epoch & 1) * kTotalCopies * MOONEP_MAX_EXPERTS;
   if (fast) {
+    int32_t *mine = totals + (k % kTotalCopies) * MOONEP_MAX_EXPERTS;
     for (int e = tid; e < (int)d.E; e += kPlanThreads)
-      if (m.base[e]) atomicAdd(totals + e, m.base[e]);
+      if (m.base[e]) atomicAdd(mine + e, m.base[e]);
     __syncthreads();
   }
   if (tid == 0) {
@@ -1682,8 +1699,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
   }
   if (k == 0) {  // zero the other buffer for the next launch (nobody uses it in this one)
     const int nxt = (epoch & 1) ^ 1;
-    int32_t *other = a.totals + nxt * MOONEP_MAX_EXPERTS;
-    for (int e = tid; e < MOONEP_MAX_EXPERTS; e += kPlanThreads) other[e] = 0;
+    int4 *other = reinterpret_cast<int4 *>(a.totals + nxt * kTotalCopies * MOONEP_MAX_EXPERTS);
+    for (int i = tid; i < kTotalCopies * MOONEP_MAX_EXPERTS / 4; i += kPlanThreads)
+      other[i] = make_int4(0, 0, 0, 0);
     __syncthreads();
     if (tid == 0) st_release(a.sync + kSyncTotTag + nxt, (int)((unsigned)epoch + kEpochStep));
   }
