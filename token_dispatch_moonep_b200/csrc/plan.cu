@@ -1207,7 +1207,9 @@ __device__ __forceinline__ void share_of(int n, int &b, int &e) {
 // The balance problem, from m.cnt, by the first NT threads of the block (the fixed
 // rule of the plan; see the file header): block scans over experts, ranks and pieces,
 // one thread per element in between.  Writes the solve state into shared memory; misc[M_CAP] != 0 if a rank
-// would pass NvS rows or the tables do not fit together (unreachable).
+// would pass NvS rows or the tables do not fit together (unreachable).  A thread's
+// loops run once or twice, so they stay rolled: the plan's code is fetched anew on
+// every launch, and unrolled copies would only lengthen that fetch.
 template <int NT, int BAR>
 __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   const int tid = threadIdx.x;
@@ -1223,7 +1225,9 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   int n_recv;
   {
     int v[4] = {0, 0, 0, 0}, ex[4], tot[4];
+#pragma unroll 1
     for (int e = eb; e < ee; e++) v[0] += m.cnt[e];
+#pragma unroll 1
     for (int h = hb; h < he; h++) {
       int ld = 0;
       for (int e = h * L; e < (h + 1) * L; e++) ld += m.cnt[e];
@@ -1234,11 +1238,13 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     }
     block_scan<4, NT, BAR>(v, ex, tot, scr);
     int run = ex[0];
+#pragma unroll 1
     for (int e = eb; e < ee; e++) {
       m.gcst[e] = run;
       run += m.cnt[e];
     }
     int ov = ex[1], df = ex[2], rf = ex[3];
+#pragma unroll 1
     for (int h = hb; h < he; h++) {
       const int ld = m.load[h];
       const int o = ld > SK ? ld - SK : 0, dd = ld < SK ? SK - ld : 0;
@@ -1270,6 +1276,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   int n_piece, padtot;
   {
     int v[2] = {0, 0}, ex[2], tot[2];
+#pragma unroll 1
     for (int e = eb; e < ee; e++) {
       const int h = home_of(d, e);
       const int c = m.cnt[e];
@@ -1294,9 +1301,11 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
       v[0] += npc;
       v[1] += A > 1 ? roundup_i(kept, A) : kept;
     }
+#pragma unroll 1
     for (int i = tid; i < n_recv; i += NT) m.rfirst[i] = m.rlast[i] = -1;  // set by its pieces
     block_scan<2, NT, BAR>(v, ex, tot, scr + 4 * kPlanWarps);
     int rp = ex[0], rk = ex[1];
+#pragma unroll 1
     for (int e = eb; e < ee; e++) {
       m.pid0[e] = rp;
       rp += m.npc[e];
@@ -1312,6 +1321,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   //     rows; a piece's expert, receiver and range (a piece that starts at its
   //     receiver's base is the receiver's first, one that ends at its end the last)
   int bad = 0;
+#pragma unroll 1
   for (int t = tid; t < E + R + n_piece; t += NT) {
     if (t < E) {
       const int e = t, h = home_of(d, e);
@@ -1350,10 +1360,12 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     int pb, pe;
     share_of<NT>(n_piece, pb, pe);
     int v[1] = {0}, ex[1], tot[1];
+#pragma unroll 1
     for (int pid = pb; pid < pe; pid++) v[0] += m.pscan[pid];
     block_scan<1, NT, BAR>(v, ex, tot, scr + 8 * kPlanWarps);
     group_sync<NT, BAR>();  // every thread has read its values before they are overwritten
     int run = ex[0];
+#pragma unroll 1
     for (int pid = pb; pid < pe; pid++) {
       const int x = m.pscan[pid];
       m.pscan[pid] = run;
@@ -1365,6 +1377,7 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
   //     receiver's rows follow its native rows in overflow-stream order), capacity,
   //     local-replica flags, remote pieces; one receiver per thread: its segment count
   int cap = 0, nrem = 0;
+#pragma unroll 1
   for (int pid = tid; pid < n_piece; pid += NT) {
     const int i = m.precv[pid], first = m.rfirst[i], dr = m.rrank[i];
     if (first < 0 || pid < first) {
@@ -1379,11 +1392,13 @@ __device__ void solve_fast(const Dims &d, const FastSmem &m) {
     if (pid - first < B) m.eflag[m.pexp[pid]] = 1;
     else nrem++;
   }
+#pragma unroll 1
   for (int i = tid; i < n_recv; i += NT) {
     const int first = m.rfirst[i], last = m.rlast[i];
     if (first < 0 || last < first || L + (last - first + 1) > E) cap = 1;
     else m.nseg[m.rrank[i]] = L + (last - first + 1);
   }
+#pragma unroll 1
   for (int h = tid; h < R; h += NT)
     if (m.ntot[h] > NvS) cap = 1;
   if (cap) atomicOr(&m.misc[M_CAP], 1);
@@ -1461,29 +1476,35 @@ __device__ __forceinline__ bool fast_row_used(const Dims &d, const FastSmem &m, 
   return m.pst[lo] <= row && row < m.pst[lo] + m.plen[lo];
 }
 
-// The user-facing tables, shared over the CTAs (every CTA holds the whole solve).
+// The user-facing tables, shared over the CTAs (every CTA holds the whole solve).  Every
+// index fits in 32 bits (R * NvS < 2^31 is checked on the host); the loops run a handful
+// of times per thread and stay rolled: the code of the plan is fetched from L2 (or
+// DRAM, after a step's kernels have streamed through it) on every launch, so its size
+// is latency.
 __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
   const Dims &d = a.d;
   const PlanPtrs &P = a.P;
   const int tid = threadIdx.x;
   const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
   const int n_piece = min(m.misc[M_NPIECE], (int)d.PMAX);
-  const int64_t gt = (int64_t)blockIdx.x * kPlanThreads + tid;
-  const int64_t stride = (int64_t)gridDim.x * kPlanThreads;
-  for (int64_t e = gt; e < E; e += stride) {
-    const int h = (int)e / L;
-    const int64_t si = (int64_t)h * E + (e - (int64_t)h * L);
+  const int gt = (int)blockIdx.x * kPlanThreads + tid;
+  const int stride = (int)gridDim.x * kPlanThreads;
+#pragma unroll 1
+  for (int e = gt; e < E; e += stride) {
+    const int h = home_of(d, e);
+    const int si = h * E + (e - h * L);
     P.f[F_EXPERT_COUNT][e] = m.cnt[e];
     P.f[F_EXP_PIECE_BEGIN][e] = m.pid0[e];
     P.f[F_EXP_PIECE_END][e] = m.pid0[e] + m.npc[e];
-    P.f[F_SEG_EXPERT][si] = (int)e;
+    P.f[F_SEG_EXPERT][si] = e;
     P.f[F_SEG_START][si] = m.nst[e];
     P.f[F_SEG_LEN][si] = m.kept[e];
     P.f[F_SEG_KIND][si] = MOONEP_SEG_NATIVE;
     P.f[F_SEG_WSLOT][si] = -1;
   }
-  for (int64_t pid = gt; pid < n_piece; pid += stride) {
-    const int i = m.precv[pid], dr = m.rrank[i], j = (int)pid - m.rfirst[i], e = m.pexp[pid];
+#pragma unroll 1
+  for (int pid = gt; pid < n_piece; pid += stride) {
+    const int i = m.precv[pid], dr = m.rrank[i], j = pid - m.rfirst[i], e = m.pexp[pid];
     const int ws = j < B ? j : -1;
     P.f[F_PIECE_EXPERT][pid] = e;
     P.f[F_PIECE_RANK][pid] = dr;
@@ -1492,24 +1513,26 @@ __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
     P.f[F_PIECE_WSLOT][pid] = ws;
     P.f[F_PIECE_OSTART][pid] = m.post[pid];
     if (j >= 0 && L + j < E) {
-      const int64_t sj = (int64_t)dr * E + L + j;
+      const int sj = dr * E + L + j;
       P.f[F_SEG_EXPERT][sj] = e;
       P.f[F_SEG_START][sj] = m.pst[pid];
       P.f[F_SEG_LEN][sj] = m.plen[pid];
       P.f[F_SEG_KIND][sj] = ws >= 0 ? MOONEP_SEG_REPLICA : MOONEP_SEG_REMOTE;
       P.f[F_SEG_WSLOT][sj] = ws;
     }
-    if (ws >= 0) P.f[F_REP_EXPERT][(int64_t)dr * B + j] = e;
+    if (ws >= 0) P.f[F_REP_EXPERT][dr * B + j] = e;
   }
-  for (int64_t h = gt; h < R; h += stride) {
+#pragma unroll 1
+  for (int h = gt; h < R; h += stride) {
     const int ld = m.load[h];
     P.f[F_RANK_LOAD][h] = ld;
     P.f[F_OVERFLOW][h] = ld > SK ? ld - SK : 0;
     P.f[F_DEFICIT][h] = ld < SK ? SK - ld : 0;
     P.f[F_N_SEG][h] = m.nseg[h];
   }
-  for (int64_t q = gt; q < (int64_t)R * E; q += stride) {  // unused segment entries
-    const int h = (int)(q / E), i = (int)(q % E);
+#pragma unroll 1
+  for (int q = gt; q < R * E; q += stride) {  // unused segment entries
+    const int h = q / E, i = q - h * E;
     if (i >= m.nseg[h]) {
       P.f[F_SEG_EXPERT][q] = -1;
       P.f[F_SEG_START][q] = 0;
@@ -1518,21 +1541,28 @@ __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
       P.f[F_SEG_WSLOT][q] = -1;
     }
   }
-  for (int64_t q = gt; q < (int64_t)R * B; q += stride) {  // free replica weight slots
-    const int h = (int)(q / B), j = (int)(q % B);
+#pragma unroll 1
+  for (int q = gt; q < R * B; q += stride) {  // free replica weight slots
+    const int h = q / B, j = q - h * B;
     if (j >= m.nseg[h] - L) P.f[F_REP_EXPERT][q] = -1;
   }
   if (d.A > 1) {  // padding rows hold no pair
     int32_t *slot_src = P.f[F_SLOT_SRC];
-    for (int64_t q = gt; q < d.R * d.NvS; q += stride)
-      if (!fast_row_used(d, m, (int)(q / d.NvS), (int)(q % d.NvS))) slot_src[q] = -1;
+    const int NvS = (int)d.NvS, rows = (int)(d.R * d.NvS);
+#pragma unroll 1
+    for (int q = gt; q < rows; q += stride) {
+      const int h = q / NvS;
+      if (!fast_row_used(d, m, h, q - h * NvS)) slot_src[q] = -1;
+    }
   }
   if (blockIdx.x == gridDim.x - 1) {  // the last chunk is the smallest: this CTA adds the rest
+#pragma unroll 1
     for (int e = tid; e < E; e += kPlanThreads) m.epos[e] = m.eflag[e];
     int *arr[1] = {m.epos};
     int tot[1];
     __syncthreads();
     block_excl_scan<1>(arr, E, m.scratch, tot);
+#pragma unroll 1
     for (int e = tid; e < E; e += kPlanThreads)
       if (m.eflag[e]) P.f[F_REPLICATED][m.epos[e]] = e;
     if (tid == 0) {
