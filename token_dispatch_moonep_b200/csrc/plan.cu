@@ -1487,7 +1487,9 @@ __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
   const int tid = threadIdx.x;
   const int E = (int)d.E, R = (int)d.R, L = (int)d.L, B = (int)d.B, SK = (int)d.SK;
   const int n_piece = min(m.misc[M_NPIECE], (int)d.PMAX);
-  const int gt = (int)blockIdx.x * kPlanThreads + tid;
+  // item i of a table goes to warp i / 32 counted across the CTAs first (warp w of CTA b
+  // is warp w * gridDim + b): the stores spread over every SM, 32 to a line
+  const int gt = ((tid >> 5) * (int)gridDim.x + (int)blockIdx.x) * 32 + (tid & 31);
   const int stride = (int)gridDim.x * kPlanThreads;
 #pragma unroll 1
   for (int e = gt; e < E; e += stride) {
@@ -1727,13 +1729,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
     // cumulative) before the flag
     st_release(a.arrive + k, epoch);
   }
-  if (k == 0) {  // zero the other buffer for the next launch (nobody uses it in this one)
+  {
+    // zero this CTA's share of the other totals buffer for the next launch (nobody uses
+    // it in this one): warps 1.. do it while warp 0 polls the arrivals.  Every CTA gets
+    // here, and the next launch reads the buffer and its tag only after this grid has
+    // completed, so no ordering inside this launch is needed.
     const int nxt = (epoch & 1) ^ 1;
     int4 *other = reinterpret_cast<int4 *>(a.totals + nxt * kTotalCopies * MOONEP_MAX_EXPERTS);
-    for (int i = tid; i < kTotalCopies * MOONEP_MAX_EXPERTS / 4; i += kPlanThreads)
-      other[i] = make_int4(0, 0, 0, 0);
-    __syncthreads();
-    if (tid == 0) st_release(a.sync + kSyncTotTag + nxt, (int)((unsigned)epoch + kEpochStep));
+    constexpr int n4 = kTotalCopies * MOONEP_MAX_EXPERTS / 4;
+    const int per = (n4 + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int z0 = (int)k * per, z1 = z0 + per < n4 ? z0 + per : n4;
+    if (warp > 0)
+      for (int i = z0 + tid - 32; i < z1; i += kPlanThreads - 32) other[i] = make_int4(0, 0, 0, 0);
+    if (k == 0 && tid == 0)
+      *((volatile int32_t *)(a.sync + kSyncTotTag + nxt)) = (int)((unsigned)epoch + kEpochStep);
   }
   int st;
   if (fast)
