@@ -1558,22 +1558,36 @@ __device__ void fast_tables(const PlanArgs &a, const FastSmem &m) {
     }
   }
   if (blockIdx.x == gridDim.x - 1) {  // the last chunk is the smallest: this CTA adds the rest
+    // the replicated experts in ascending order: a ballot per warp of 32 experts, the
+    // warps' counts added up in shared memory
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = lanemask_lt();
+    int carry = 0;
 #pragma unroll 1
-    for (int e = tid; e < E; e += kPlanThreads) m.epos[e] = m.eflag[e];
-    int *arr[1] = {m.epos};
-    int tot[1];
-    __syncthreads();
-    block_excl_scan<1>(arr, E, m.scratch, tot);
-#pragma unroll 1
-    for (int e = tid; e < E; e += kPlanThreads)
-      if (m.eflag[e]) P.f[F_REPLICATED][m.epos[e]] = e;
+    for (int e0 = 0; e0 < E; e0 += kPlanThreads) {
+      const int e = e0 + tid;
+      const bool f = e < E && m.eflag[e];
+      const uint32_t b = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) m.scratch[warp] = __popc(b);
+      __syncthreads();
+      int before = carry, all = 0;
+#pragma unroll
+      for (int w = 0; w < kPlanWarps; w++) {
+        const int x = m.scratch[w];
+        before += w < warp ? x : 0;
+        all += x;
+      }
+      if (f) P.f[F_REPLICATED][before + __popc(b & lt)] = e;
+      carry += all;
+      __syncthreads();
+    }
     if (tid == 0) {
       const int n_remote = m.misc[M_NREMOTE];
       int32_t *sc = P.f[F_SCALARS];
       sc[S_N_PIECE] = n_piece;
       sc[S_N_REMOTE] = n_remote;
       sc[S_N_LOCAL] = n_piece - n_remote;
-      sc[S_N_REPLICATED] = tot[0];
+      sc[S_N_REPLICATED] = carry;
       sc[S_BAD] = 0;
       sc[5] = sc[6] = sc[7] = 0;
       if (d.mode == MOONEP_MODE_TRAIN && n_remote > 0) set_status(a.status, MOONEP_DEV_BUDGET);
