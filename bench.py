@@ -86,7 +86,8 @@ def hbm_peak():
 
 def ncu_traffic(workload, maxvio, seed):
     """Per-kernel DRAM bytes per launch from the committed ncu summary, if it was taken on
-    this workload (name, maxvio, seed) and the kernel's source has not changed since."""
+    this workload (name, maxvio, seed) and neither the kernel's source nor the shared
+    header has changed since."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     out = {}
@@ -107,7 +108,10 @@ def ncu_traffic(workload, maxvio, seed):
         parts = dict(kv.split("=", 1) for kv in ln.split())
         same_case = (parts.get("workload") == workload and parts.get("seed") == str(seed)
                      and abs(float(parts.get("maxvio", "nan")) - maxvio) < 1e-9)
-        if same_case and src_hash.get(parts.get("source")) == parts.get("sha"):
+        same_src = (src_hash.get(parts.get("source")) == parts.get("sha") and
+                    parts.get("header_sha", src_hash.get("moonep_internal.cuh"))
+                    == src_hash.get("moonep_internal.cuh"))
+        if same_case and same_src:
             out[parts["kernel"]] = float(parts["bytes_per_launch"])
     return out
 

@@ -119,3 +119,29 @@ def test_reference_line_carries_the_gpu_arm_config():
     _, alpha, mv = make_routing(w.R, w.E, w.K, w.S, w.maxvio[0], 0)
     assert d["config"] == bench.workload_config(w, mv, alpha, 1)
     assert d["cpu_baseline"]["cores"] == bench.host_cores()
+
+
+def test_profiles_name_the_current_sources():
+    """Every ncu summary under profiles/ states the sha256 (16 hex digits) of the sources
+    it was captured on; each stated hash is that of the file as it is now."""
+    import glob
+    import hashlib
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    csrc = os.path.join(root, "token_dispatch_moonep_b200", "csrc")
+    now = {f: hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()[:16]
+           for f in os.listdir(csrc) if f.endswith((".cu", ".cuh"))}
+    files = sorted(glob.glob(os.path.join(root, "profiles", "*.md")))
+    assert files
+    for path in files:
+        text = open(path).read()
+        stated = re.findall(r"`csrc/([\w.]+)` ([0-9a-f]{16})", text)
+        assert stated, f"{os.path.basename(path)} names no source hash"
+        for name, h in stated:
+            assert now.get(name) == h, f"{os.path.basename(path)}: {name} is {now.get(name)}, not {h}"
+    for ln in open(os.path.join(root, "profiles", "ncu_traffic.txt")):
+        if ln.startswith("#") or not ln.strip():
+            continue
+        parts = dict(kv.split("=", 1) for kv in ln.split())
+        assert now[parts["source"]] == parts["sha"]
+        assert now["moonep_internal.cuh"] == parts["header_sha"]
