@@ -11,16 +11,24 @@
 // plan_kernel (chunks <= co-resident CTAs): CTA k owns chunk k of 512*ppt pairs.
 //   count    warp-private per-expert counters in shared memory give every pair its
 //            stable rank among the chunk's pairs of the same expert (lanes with
-//            equal ids found with match.any: a hot expert costs one counter update
-//            per warp step, no atomics); the chunk histogram is published as a
-//            uint16 row with one release store of an arrival flag.
-//   gather   once every flag shows this launch's epoch (warp 0 polls), each CTA
-//            sums all rows: the expert counts, and the counts of the chunks
-//            before its own (its pairs' base offsets).
+//            equal ids found by one ballot per bit of the id: a fixed cost however
+//            many distinct ids a warp holds, no atomics).
+//   publish  the chunk's counts are added by atomics into one of 16 spread copies
+//            of the expert totals (a buffer per epoch parity, zeroed by the launch
+//            before), the histogram is stored as a uint16 row, and one release
+//            store of an arrival flag publishes both.
+//   gather   once every flag shows this launch's epoch (warp 0 polls), warps 0..7
+//            read the totals while warps 8..15 sum the rows before or after the
+//            chunk (the nearer end) into its pairs' base offsets.  The first launch
+//            on a workspace has no zeroed totals and sums every row instead.
 //   solve    each CTA solves the O(E + R) problem itself with block scans; all
 //            CTAs reach the same tables, so nobody waits for anybody again.
 //   place    each CTA places its own pairs straight from its shared memory.
-//   tables   each CTA writes its share of the user-facing plan tables.
+//   tables   the user-facing tables, spread over the warps of all CTAs; the last
+//            CTA lists the replicated experts.
+// The kernel's code is fetched anew on every launch (inside a step the data kernels
+// have streamed gigabytes through L2 since the last plan), so loops that run once or
+// twice per thread stay rolled and the table phase keeps to 32-bit indices.
 // plan_multichunk_kernel (larger batches): CTA 0 solves, CTAs 1..W are workers
 //            with several chunks each; workers keep stable ranks in the workspace,
 //            the solver turns the histograms into per-chunk bases and publishes the
@@ -221,6 +229,7 @@ __device__ void column_sums(const int32_t *hist, int E, int64_t nrows, int *out,
 // k*ch + w*32*ppt + j*32 + l.  ev[j]: expert id, -1 bad id, -2 past the end.
 // kU16: the histogram row is written as uint16 (a chunk holds at most 8192 pairs).
 // chunk_tot (may be null): the chunk's count of each expert, in shared memory.
+// The caller puts a block barrier after the call before wh is written again.
 template <bool kU16>
 __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *wh,
                                             int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread],
@@ -285,7 +294,6 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
 #pragma unroll
   for (int j = 0; j < kPairsPerThread; j++)
     if (ev[j] >= 0) rk[j] += myh[ev[j]];
-  __syncthreads();  // wh is reused by the caller
   return bad;
 }
 
@@ -1427,9 +1435,12 @@ __device__ int gather_split(const PlanArgs &a, int64_t k, int epoch, const int32
   if (m.misc[M_STATE]) return kStTimeout;
   if (warp < kPlanWarps / 2) {
     constexpr int NT = kPlanThreads / 2;
+    // the first bad-id mark is loaded with the totals (one L2 round trip for both)
+    const bool has_mark = tid < a.nc;
+    const int mark = has_mark ? __ldcg(a.badmark + tid) : 0;
     for (int e = tid; e < E; e += NT) m.cnt[e] = total_of(totals, e);
-    bool bad = false;
-    for (int64_t c = tid; c < a.nc; c += NT) bad |= __ldcg(a.badmark + c) == epoch;
+    bool bad = has_mark && mark == epoch;
+    for (int64_t c = tid + NT; c < a.nc; c += NT) bad |= __ldcg(a.badmark + c) == epoch;
     if (bad) atomicOr(&m.misc[M_STATE], kStBad);
     group_sync<NT, 1>();
     if (m.misc[M_STATE] == 0) solve_fast<NT, 1>(a.d, m);
@@ -1717,7 +1728,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
     tag1 = *((volatile int32_t *)(a.sync + kSyncTotTag + 1));
   }
   int ev[kPairsPerThread], rk[kPairsPerThread];
-  const bool bad = __syncthreads_or(count_chunk<true>(a, k, m.tmp, ev, rk, m.base));
+  const bool bad_here = count_chunk<true>(a, k, m.tmp, ev, rk, m.base);
   if (tid == 0) {
     const int e = (int)((unsigned)gen_v + kEpochStep);
     s_epoch = e;
@@ -1725,7 +1736,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
     // launch before (else: first use of the workspace, or it ran another kernel)
     s_fast = ((e & 1) ? tag1 : tag0) == e;
   }
-  __syncthreads();
+  const bool bad = __syncthreads_or(bad_here);
   const int epoch = s_epoch;
   const bool fast = s_fast;
   int32_t *totals = a.totals + (epoch & 1) * kTotalCopies * MOONEP_MAX_EXPERTS;
