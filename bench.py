@@ -12,7 +12,8 @@ Metric (headline): dispatch+combine HBM GB/s = algorithmic bytes of the two
 kernels / their CUDA-event time, plus plan µs per layer.  ms_per_step comes from
 K steps with events only around them (kernels overlap their launch gaps as in
 use); the per-kernel times, the metric and the roofline from a second pass of
-K steps with an event after every kernel.
+K steps with an event after every kernel; `b2b_ms` per data kernel from ten
+launches in a row between two events (no event between launches).
 Default workload: R=8 ranks, E=256 experts, K=8, S=4096 tokens/rank, H=7168,
 maxvio 0.2, replica budget 32 (training).  The default run then adds, on the
 same line: `sweep` — the forward layer (plan + dispatch + combine) of the same
@@ -359,6 +360,29 @@ def time_steps(layer, steps, warmup, barrier=None, ops=None):
            for i, (name, _) in enumerate(ops)}
     st = int(layer.status.item())
     return total_ms, per, clocks, st
+
+
+def time_back_to_back(layer, n=10, ops=None):
+    """Each data kernel launched n times in a row between two events (after two untimed
+    launches): its average launch duration without an event between launches, which
+    otherwise adds a few microseconds to every launch.  The plan is left out: its
+    latency inside the step is what counts."""
+    torch = layer.torch
+    out = {}
+    for name, fn in (ops or layer.ops()):
+        if name == "plan":
+            continue
+        fn()
+        fn()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / n
+    return out
 
 
 def time_e2e(layer, steps):
@@ -821,6 +845,11 @@ def main():
         avg = sum(ts) / len(ts)
         kern[name] = {"ms": avg, "bytes": b[name], "GBs": b[name] / (avg * 1e-3) / 1e9,
                       "frac": b[name] / (avg * 1e-3) / 1e9 / peak, "share": sum(ts) / per_total}
+    b2b = time_back_to_back(layer)
+    names = sorted(b2b)
+    for name, ms in zip(names, max_over_ranks(pg, [b2b[n] for n in names], device)):
+        kern[name].update({"b2b_ms": ms, "b2b_GBs": b[name] / (ms * 1e-3) / 1e9,
+                           "b2b_frac": b[name] / (ms * 1e-3) / 1e9 / peak})
     kern["plan"].pop("frac")
     # the plan is a latency: its per-layer figure is the median over the steps
     kern["plan"]["ms_mean"] = kern["plan"]["ms"]
