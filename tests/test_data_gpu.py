@@ -390,7 +390,7 @@ def test_chained_calls_without_host_syncs():
     w = normal_bf16((E, P), seed=21, stream=4)
     home0 = normal_bf16((E, P), seed=21, stream=5)
     arena, ws, st = me.alloc_plan(cfg)
-    arena2, ws2, _ = me.alloc_plan(cfg)
+    arena2, _, _ = me.alloc_plan(cfg)
     idx1_d, idx2_d = to_dev(idx1.ravel().astype(np.int32)), to_dev(idx2.ravel().astype(np.int32))
     x_d, g_d, dout_d, w_d = to_dev(x), to_dev(g.ravel()), to_dev(dout), to_dev(w)
     home = to_dev(home0)
@@ -408,7 +408,7 @@ def test_chained_calls_without_host_syncs():
     me.moonep_combine_backward(cfg, arena, dout_d, recv, g_d, dy, dg, st)
     me.moonep_dispatch_backward(cfg, arena, dy, dx, st)
     me.moonep_reduce_grad(cfg, arena, rep_w, home, P, st)  # replica "grads" = the prefetched weights
-    me.moonep_plan(cfg, idx2_d, arena2, ws2, st)
+    me.moonep_plan(cfg, idx2_d, arena2, ws, st)             # same workspace: the steady-state path
     me.moonep_dispatch(cfg, arena2, out, recv, st)          # second layer reads the first's output
     torch.cuda.synchronize()
     assert int(st.item()) & ~me.DEV_BUDGET == 0
