@@ -385,6 +385,33 @@ def time_back_to_back(layer, n=10, ops=None):
     return out
 
 
+def host_cost(layer, n=500):
+    """Host time of one enqueue through the C ABI (ctypes call with pointers already
+    marshalled; the GPU work queues up behind), in µs per call: the library's argument
+    checks, its cached launch facts and the launch itself."""
+    import ctypes
+    torch, me, c = layer.torch, layer.me, layer.cfg
+    lib = me._lib
+    s = torch.cuda.current_stream().cuda_stream
+    cp = ctypes.byref(c)
+    calls = {
+        "plan": lambda: lib.moonep_plan(cp, layer.idx.data_ptr(), layer.arena.data_ptr(),
+                                        layer.ws.data_ptr(), layer.status.data_ptr(), s),
+        "dispatch": lambda: lib.moonep_dispatch(cp, layer.arena.data_ptr(), layer.x.data_ptr(),
+                                                layer.recv.data_ptr(), layer.status.data_ptr(), s),
+    }
+    out = {}
+    for name, fn in calls.items():
+        torch.cuda.synchronize()
+        fn()
+        t0 = time.perf_counter()
+        for _ in range(n):
+            fn()
+        out[name] = (time.perf_counter() - t0) / n * 1e6
+        torch.cuda.synchronize()
+    return out
+
+
 def time_e2e(layer, steps):
     """The same steps through the public API from host memory, pipelined as a user would:
     step s+1's inputs are copied in from pinned host memory (H2D stream) and step s-1's
@@ -845,6 +872,7 @@ def main():
         avg = sum(ts) / len(ts)
         kern[name] = {"ms": avg, "bytes": b[name], "GBs": b[name] / (avg * 1e-3) / 1e9,
                       "frac": b[name] / (avg * 1e-3) / 1e9 / peak, "share": sum(ts) / per_total}
+    host_us = host_cost(layer, n=200 if w.name == DEFAULT_WORKLOAD else 500)
     b2b = time_back_to_back(layer)
     names = sorted(b2b)
     for name, ms in zip(names, max_over_ranks(pg, [b2b[n] for n in names], device)):
@@ -905,6 +933,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
+            "host_us_per_call": host_us,
             "clocks": clocks,
             "sweep": sweep,
             "decode": decode,
