@@ -130,7 +130,11 @@ MOONEP_API int64_t moonep_nvs(const moonep_config_t *cfg);
 MOONEP_API size_t moonep_plan_bytes(const moonep_config_t *cfg);
 
 /* Bytes of scratch the plan needs (device, 256-byte aligned base); 0 if invalid.
- * Contents need no initialisation and are meaningless between calls. */
+ * Contents need no initialisation: any bytes are valid before a call.  A call
+ * leaves state for the next call on the same workspace (a generation word and
+ * expert totals zeroed ahead, at fixed offsets, for any config); a call that
+ * finds none (the first on a workspace) takes a slower gather with the same
+ * result.  Calls that share a workspace must be ordered on the GPU. */
 MOONEP_API size_t moonep_workspace_bytes(const moonep_config_t *cfg);
 
 /* Plan ("Moonshot AI Open-Sources MoonEP", S x K and replica-slot paragraphs;
@@ -183,14 +187,15 @@ MOONEP_API moonep_status_t moonep_plan_static(const moonep_config_t *cfg, const 
                                               moonep_stream_t stream);
 
 /* Diagnostics for the bounded in-kernel waits (process-wide, host-side).
- * The plan is one cooperative launch whose CTAs wait for each other twice;
+ * The plan is one cooperative launch whose CTAs wait for every CTA's arrival
+ * (batches of more chunks than co-resident CTAs also wait for the solving CTA);
  * reduce_grad's pipeline waits on shared-memory barriers for its bulk copies.
  * Each wait gives up after `limit_ns` nanoseconds (default 200 ms) and sets
  * MOONEP_DEV_TIMEOUT instead of hanging (a timed-out plan is invalid:
  * slot_of = -1).  `phantom_arrivals` (tests only, 0..32) forces the timeout:
- * the plan's solving CTA also waits for that many arrivals that no CTA ever
- * makes, and each reduce_grad CTA's first stage expects 16 bytes per phantom
- * arrival more than its copies deliver. */
+ * the plan's CTAs also wait for that many arrivals that no CTA ever makes, and
+ * each reduce_grad CTA's first stage expects 16 bytes per phantom arrival more
+ * than its copies deliver. */
 MOONEP_API moonep_status_t moonep_debug_set_wait(int64_t limit_ns, int32_t phantom_arrivals);
 
 /* Fill `out` with device pointers into `plan_arena` (pure host arithmetic). */
