@@ -12,6 +12,7 @@
 // (one bf16 per lane) path.
 #include <cuda_bf16.h>
 
+#include <mutex>
 #include <utility>
 
 #include "moonep_internal.cuh"
@@ -198,17 +199,23 @@ combine_vec_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict_
 }
 
 // K <= KMAX: the K rows of a column chunk are loaded before any arithmetic, so
-// a warp keeps K*U 16-byte loads in flight.
+// a warp keeps K*U 16-byte loads in flight.  A warp's unit is a token, or with
+// split = 1 one half of its columns [c0, c0 + cl) (small batches: twice the units,
+// so the last wave of warps is not left half empty).
 template <int U, int KMAX>
 __global__ void __launch_bounds__(kThreads)
 combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restrict__ y,
                      const float *__restrict__ gates, uint4 *__restrict__ out, int64_t T, int K,
-                     int64_t nvec, int64_t nrows, int32_t *status) {
+                     int64_t nvec, int split, int64_t cl, int64_t nrows, int32_t *status) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t warp_g = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerBlock;
-  for (int64_t t = warp_g; t < T; t += nwarps) {
+  const int64_t nunits = T << split;
+  for (int64_t w = warp_g; w < nunits; w += nwarps) {
+    const int64_t t = w >> split;
+    const int64_t c0 = (w - (t << split)) * cl;
+    const int64_t c1 = c0 + cl < nvec ? c0 + cl : nvec;
     const int my_slot = load_slot(slot_of, t, K, nrows, status);
     const float my_w = lane < K ? (gates ? __ldg(gates + t * K + lane) : 1.f) : 0.f;
     int rows[KMAX];
@@ -218,15 +225,15 @@ combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restric
       rows[k] = __shfl_sync(0xffffffffu, my_slot, k);
       ws[k] = __shfl_sync(0xffffffffu, my_w, k);
     }
-    for (int64_t v0 = 0; v0 < nvec; v0 += 32 * U) {
+    for (int64_t v0 = c0; v0 < c1; v0 += 32 * U) {
       uint4 q[KMAX][U];
 #pragma unroll
       for (int k = 0; k < KMAX; k++)
 #pragma unroll
         for (int u = 0; u < U; u++) {
           const int64_t v = v0 + u * 32 + lane;
-          q[k][u] = (rows[k] >= 0 && v < nvec) ? __ldcs(y + (int64_t)rows[k] * nvec + v)
-                                               : make_uint4(0, 0, 0, 0);
+          q[k][u] = (rows[k] >= 0 && v < c1) ? __ldcs(y + (int64_t)rows[k] * nvec + v)
+                                             : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
       for (int u = 0; u < U; u++) {
@@ -244,7 +251,7 @@ combine_vec_k_kernel(const int32_t *__restrict__ slot_of, const uint4 *__restric
             acc[2 * i + 1] = __fmaf_rn(ws[k], bf16_hi(wd[i]), acc[2 * i + 1]);
           }
         }
-        if (v < nvec) {
+        if (v < c1) {
           uint4 o;
           o.x = pack_bf16x2(acc[0], acc[1]);
           o.y = pack_bf16x2(acc[2], acc[3]);
@@ -584,7 +591,7 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
   __syncthreads();
 
   // Both roles walk the same sequence: units u = blockIdx.x + j * gridDim.x,
-  // each split into ng = max(1, ceil(local pieces / 2)) stages, stage k of the
+  // each split into stages_of(local pieces, kSlots) stages, stage k of the
   // sequence in buffer k % kStages.
   if (warp == kConsumerWarps) {  // ------------------------------- producer
     if (lane != 0) return;
@@ -935,6 +942,47 @@ reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t 
 
 int num_sms() { return current_sm_count(); }
 
+// Co-resident CTAs per SM of reduce_grad_bulk_kernel, -1 on a CUDA error.  Its shared
+// memory limit is a per-context function attribute: it is raised once per CUDA context
+// and the occupancy answer is kept with the context id, per device.
+int rg_blocks_per_sm() {
+  static std::mutex mu;
+  static unsigned long long ctx_of[kMaxDevices];
+  static int per_sm_of[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return -1;
+  }
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lk(mu);
+  if (ctx != 0 && ctx_of[dev] == ctx && per_sm_of[dev] > 0) return per_sm_of[dev];
+  int per_sm = 0;
+  if (cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           rg::kSmem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_grad_bulk_kernel, rg::kThreadsRg,
+                                                    rg::kSmem) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    return -1;
+  }
+  ctx_of[dev] = ctx;
+  per_sm_of[dev] = per_sm;
+  return per_sm;
+}
+
+// combine_vec_k_kernel's units: whole tokens, or column halves (split = 1) when the
+// tokens would fill fewer than eight waves of the resident warps (two 8-warp CTAs per
+// SM); a half is a multiple of 64 vectors, the kernel's column step.
+struct CombineSplit {
+  int split;
+  int64_t cl;
+};
+CombineSplit combine_split(int64_t T, int64_t nvec) {
+  const int64_t resident = (int64_t)num_sms() * 2 * kWarpsPerBlock;
+  if (T >= 8 * resident || nvec < 128) return {0, nvec};
+  return {1, ((nvec + 1) / 2 + 63) / 64 * 64};
+}
+
 unsigned token_grid(int64_t T) {
   int64_t blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
   const int64_t cap = (int64_t)num_sms() * 64;
@@ -987,9 +1035,10 @@ extern "C" moonep_status_t moonep_combine(const moonep_config_t *cfg, const void
   cudaStream_t st = to_cuda(stream);
   const int64_t nrows = d.R * d.NvS;
   if (d.H % 8 == 0 && aligned16(y) && aligned16(out) && d.K <= 8) {
-    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
+    const CombineSplit cs = combine_split(T, d.H / 8);
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T << cs.split), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
-        T, (int)d.K, d.H / 8, nrows, dev_status);
+        T, (int)d.K, d.H / 8, cs.split, cs.cl, nrows, dev_status);
   } else if (d.H % 8 == 0 && aligned16(y) && aligned16(out)) {
     launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(y), gates, reinterpret_cast<uint4 *>(out),
@@ -1046,14 +1095,8 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
   cudaStream_t st = to_cuda(stream);
   if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
     // bulk copies need 16-byte aligned rows: P % 8 == 0 and aligned bases
-    if (cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             rg::kSmem) != cudaSuccess)
-      return MOONEP_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_grad_bulk_kernel,
-                                                      rg::kThreadsRg, rg::kSmem) != cudaSuccess ||
-        per_sm < 1)
-      return MOONEP_ERR_CUDA;
+    const int per_sm = rg_blocks_per_sm();
+    if (per_sm < 1) return MOONEP_ERR_CUDA;
     const rg::Tables t{P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN],
                        P.f[F_EXP_PIECE_END], P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT],
                        (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX, debug_wait_limit_ns(),
@@ -1084,9 +1127,10 @@ extern "C" moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
   const int64_t nrows = d.R * d.NvS;
   // the combine kernels with unit weights: fmaf(1, y, acc) rounds like acc + y
   if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx) && d.K <= 8) {
-    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
+    const CombineSplit cs = combine_split(T, d.H / 8);
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T << cs.split), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
-        reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, nrows, dev_status);
+        reinterpret_cast<uint4 *>(dx), T, (int)d.K, d.H / 8, cs.split, cs.cl, nrows, dev_status);
   } else if (d.H % 8 == 0 && aligned16(d_recv) && aligned16(dx)) {
     launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         P.f[F_SLOT_OF], reinterpret_cast<const uint4 *>(d_recv), nullptr,
@@ -1189,14 +1233,16 @@ extern "C" moonep_status_t moonep_combine_via_buffer(const moonep_config_t *cfg,
       P.f[F_SLOT_OF], comm_index, reinterpret_cast<const uint4 *>(y), reinterpret_cast<uint4 *>(comm),
       N, d.H / 8, nrows);
   // and the source ranks combine from the communication buffer
-  if (d.K <= 8)
-    launch((combine_vec_k_kernel<2, 8>), token_grid(T), kThreads, 0, st,
+  if (d.K <= 8) {
+    const CombineSplit cs = combine_split(T, d.H / 8);
+    launch((combine_vec_k_kernel<2, 8>), token_grid(T << cs.split), kThreads, 0, st,
         comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
-        (int)d.K, d.H / 8, nrows, dev_status);
-  else
+        (int)d.K, d.H / 8, cs.split, cs.cl, nrows, dev_status);
+  } else {
     launch(combine_vec_kernel<4>, token_grid(T), kThreads, 0, st,
         comm_index, reinterpret_cast<const uint4 *>(comm), gates, reinterpret_cast<uint4 *>(out), T,
         (int)d.K, d.H / 8, nrows, dev_status);
+  }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
