@@ -228,12 +228,14 @@ __device__ void column_sums(const int32_t *hist, int E, int64_t nrows, int *out,
 // chunk's pairs of the same expert.  Pair of (warp w, step j, lane l) is
 // k*ch + w*32*ppt + j*32 + l.  ev[j]: expert id, -1 bad id, -2 past the end.
 // kU16: the histogram row is written as uint16 (a chunk holds at most 8192 pairs).
-// chunk_tot (may be null): the chunk's count of each expert, in shared memory.
+// pre(): run by every thread once the loads are issued, before the first barrier.
+// tot(): after that barrier, where to add the chunk's count of each expert by
+// atomics (null: nowhere).
 // The caller puts a block barrier after the call before wh is written again.
-template <bool kU16>
+template <bool kU16, class Pre, class Tot>
 __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *wh,
                                             int (&ev)[kPairsPerThread], int (&rk)[kPairsPerThread],
-                                            int *chunk_tot = nullptr) {
+                                            Pre pre, Tot tot) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = (int)a.d.E, ppt = a.ppt;
   for (int i = tid; i < kPlanWarps * E; i += kPlanThreads) wh[i] = 0;
@@ -252,7 +254,9 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
     }
     ev[j] = e;
   }
+  pre();
   __syncthreads();
+  int32_t *const tot_dst = tot();
   int *myh = wh + warp * E;
   const uint32_t lt = lanemask_lt();
   // lanes holding the same id: one ballot per bit of the key id + 2 (id -1: a bad id,
@@ -288,7 +292,7 @@ __device__ __forceinline__ bool count_chunk(const PlanArgs &a, int64_t k, int *w
       reinterpret_cast<uint16_t *>(a.hist)[k * E + e] = (uint16_t)acc;
     else
       a.hist[k * E + e] = acc;
-    if (chunk_tot) chunk_tot[e] = acc;
+    if (tot_dst && acc) atomicAdd(tot_dst + e, acc);
   }
   __syncthreads();
 #pragma unroll
@@ -796,7 +800,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_multichunk_kernel(PlanArgs 
   int epoch = 0;
   bool have_epoch = false;
   for (int64_t k = wk; k < a.nc; k += W) {
-    const bool bad = __syncthreads_or(count_chunk<false>(a, k, smem, ev, rk));
+    const bool bad = __syncthreads_or(count_chunk<false>(
+        a, k, smem, ev, rk, [] {}, []() -> int32_t * { return nullptr; }));
     if (!have_epoch) {
       if (tid == 0) s_epoch = (int)((unsigned)gen_v + kEpochStep);
       __syncthreads();
@@ -1728,24 +1733,26 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a, FusedArg
     tag1 = *((volatile int32_t *)(a.sync + kSyncTotTag + 1));
   }
   int ev[kPairsPerThread], rk[kPairsPerThread];
-  const bool bad_here = count_chunk<true>(a, k, m.tmp, ev, rk, m.base);
-  if (tid == 0) {
-    const int e = (int)((unsigned)gen_v + kEpochStep);
-    s_epoch = e;
-    // the totals buffer of this epoch's parity was zeroed for exactly this epoch by the
-    // launch before (else: first use of the workspace, or it ran another kernel)
-    s_fast = ((e & 1) ? tag1 : tag0) == e;
-  }
-  const bool bad = __syncthreads_or(bad_here);
+  // the epoch, once the ids' loads are in flight; the chunk's counts go by atomics
+  // into copy k % 16 of this epoch's totals buffer as soon as they are summed, if that
+  // buffer was zeroed for exactly this epoch by the launch before (else: first use of
+  // the workspace, or it ran another kernel)
+  const bool bad = __syncthreads_or(count_chunk<true>(
+      a, k, m.tmp, ev, rk,
+      [&] {
+        if (tid == 0) {
+          const int e = (int)((unsigned)gen_v + kEpochStep);
+          s_epoch = e;
+          s_fast = ((e & 1) ? tag1 : tag0) == e;
+        }
+      },
+      [&]() -> int32_t * {
+        return s_fast ? a.totals + ((s_epoch & 1) * kTotalCopies + k % kTotalCopies) * MOONEP_MAX_EXPERTS
+                      : nullptr;
+      }));
   const int epoch = s_epoch;
   const bool fast = s_fast;
   int32_t *totals = a.totals + (epoch & 1) * kTotalCopies * MOONEP_MAX_EXPERTS;
-  if (fast) {
-    int32_t *mine = totals + (k % kTotalCopies) * MOONEP_MAX_EXPERTS;
-    for (int e = tid; e < (int)d.E; e += kPlanThreads)
-      if (m.base[e]) atomicAdd(mine + e, m.base[e]);
-    __syncthreads();
-  }
   if (tid == 0) {
     if (bad) set_status(a.status, MOONEP_DEV_BAD_EXPERT_ID);
     a.badmark[k] = bad ? epoch : ~epoch;
