@@ -560,15 +560,49 @@ def fused_pass(layer, steps, warmup):
             "fused_status": st}, clocks
 
 
+def graph_pass(layer, layers=10, replays=4):
+    """The forward layer (plan, dispatch, combine) as a serving loop would run it: `layers`
+    layers captured in one CUDA graph (the plan's launch epoch advances on every replay),
+    replayed `replays` times between two events; (µs per layer, device status)."""
+    torch = layer.torch
+    ops = layer.ops(forward_only=True)
+    layer.status.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _, fn in ops:  # first calls (cached launch facts) before the capture
+            fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(layers):
+            for _, fn in ops:
+                fn()
+    with torch.cuda.stream(s):
+        g.replay()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(replays):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (layers * replays)
+    del g
+    return us, int(layer.status.item())
+
+
 def decode_runs(device, steps, warmup, maxvios=(1.0, 20.0), seed=0):
     """The 64-rank inference workload: plan + dispatch + combine µs per maxvio, as three
-    calls and as the one-launch fused layer."""
+    calls, as the same three calls replayed from a CUDA graph of ten layers, and as the
+    one-launch fused layer."""
     w = WORKLOADS[DECODE_WORKLOAD]
     layer = Layer(w, maxvios[0], seed, device, with_backward=False, host_inputs=False)
     out, clocks = [], []
     for mv in maxvios:
         layer.set_routing(mv, seed)
         r, c = forward_pass(layer, steps, warmup)
+        r["graph_layer_us"], r["graph_status"] = graph_pass(layer)
         fr, fc = fused_pass(layer, steps, warmup)
         r.update(fr)
         out.append(r)
