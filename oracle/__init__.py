@@ -33,6 +33,11 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
 * ``prefetch_weight`` — every local replica slot holds its expert's weights
   bit for bit, every other slot is untouched; closed form for all tokens on
   one expert.
+* ``segment_weights`` — the weights each segment computes with: replica pieces
+  their local slot, native segments and remote pieces the home expert ("Moonshot
+  AI Open-Sources MoonEP", replica-slot paragraph: reads past the budget go to
+  the home rank).  Pinned by the worked example by hand, and against the piece
+  and replica-slot tables (a route that does not read the segment tables).
 """
 from __future__ import annotations
 
@@ -107,6 +112,8 @@ def _L():
         lib.orc_dispatch_backward_tokens.restype = None
         lib.orc_prefetch_weight.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
         lib.orc_prefetch_weight.restype = None
+        lib.orc_segment_weights.argtypes = [cp, vp, vp, vp, ctypes.c_int64, vp, vp]
+        lib.orc_segment_weights.restype = None
         lib.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.orc_f32_to_bf16.restype = ctypes.c_uint16
         lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -239,6 +246,21 @@ def prefetch_weight(cfg: Config, tables: Dict[str, np.ndarray], w: np.ndarray,
     _L().orc_prefetch_weight(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(ww), _p(rep_w),
                              ww.shape[-1])
     return rep_w
+
+
+def segment_weights(cfg: Config, tables: Dict[str, np.ndarray], W: int
+                    ) -> Tuple[np.ndarray, np.ndarray]:
+    """The weight matrix of every segment-table entry: (buf, off), both [R, E]; buf 0 is
+    the home weights [E, W], 1 the replica slots [R, budget, W], -1 none; off the first
+    element of the matrix in that buffer, -1 for none."""
+    R, E = cfg.R, cfg.E
+    se = _c(tables["seg_expert"], np.int32)
+    sk = _c(tables["seg_kind"], np.int32)
+    sw = _c(tables["seg_wslot"], np.int32)
+    buf = np.empty((R, E), np.int32)
+    off = np.empty((R, E), np.int64)
+    _L().orc_segment_weights(ctypes.byref(cfg), _p(se), _p(sk), _p(sw), int(W), _p(buf), _p(off))
+    return buf, off
 
 
 def f32_to_bf16(v: float) -> int:

@@ -407,6 +407,33 @@ void orc_dispatch_backward_tokens(const orc_config *c, const int32_t *slot_of,
   }
 }
 
+/* -------------------------------------------------------- segment_weights --- */
+/* The weight matrix each entry of the per-rank segment tables computes with: a
+   native segment reads its home expert's weights w[e]; a replica piece reads its
+   rank's local slot rep_w[d][j]; a remote piece (no local slot, past the budget)
+   reads the home weights w[e] on the home rank; an unused entry reads nothing.
+   buf[q] = 0 for w, 1 for rep_w, -1 for none; off[q] = the matrix's first
+   element in that buffer (row * W), -1 for none.  q = d * E + i. */
+void orc_segment_weights(const orc_config *c, const int32_t *seg_expert, const int32_t *seg_kind,
+                         const int32_t *seg_wslot, int64_t W, int32_t *buf, int64_t *off) {
+  const int64_t R = c->R, E = c->E, B = c->budget;
+  for (int64_t d = 0; d < R; d++) {
+    for (int64_t i = 0; i < E; i++) {
+      const int64_t q = d * E + i;
+      if (seg_kind[q] == KIND_REPLICA) {
+        buf[q] = 1;
+        off[q] = (d * B + seg_wslot[q]) * W;
+      } else if (seg_kind[q] == KIND_NATIVE || seg_kind[q] == KIND_REMOTE) {
+        buf[q] = 0;
+        off[q] = (int64_t)seg_expert[q] * W;
+      } else {
+        buf[q] = -1;
+        off[q] = -1;
+      }
+    }
+  }
+}
+
 /* --------------------------------------------------------- prefetch_weight --- */
 /* For every piece with a local weight slot: rep_w[rank][slot] = w[expert] (W elements).
    rep_w is [R, budget, W]; w is [E, W]. */

@@ -4,7 +4,8 @@ Each case plants one mistake in a scratch copy of oracle/moonep_oracle.c
 (wrong keep/overflow cut, wrong receiver order, wrong layout, wrong weight
 slot, a dropped term, a missing gate, a skipped replica, ignored alignment,
 truncating instead of rounding, reversed per-expert order, a half dot
-product), builds it with gcc, and runs the pin tests against it: at least one
+product, a remote piece or a replica slot mapped to the wrong weights),
+builds it with gcc, and runs the pin tests against it: at least one
 pin must fail.  Everything runs on the CPU.
 """
 import os
@@ -39,6 +40,9 @@ MUTANTS = {
                               "rep_w[slot * W + q] = w[(int64_t)((piece_expert[i] + 1) % c->E) * W + q];"),
     "half_dot_product": ("dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);",
                          "if (h % 2 == 0) dot += (double)g * (double)orc_bf16_to_f32(y[row * H + h]);"),
+    "remote_piece_reads_replica_slot": ("} else if (seg_kind[q] == KIND_NATIVE || seg_kind[q] == KIND_REMOTE) {",
+                                        "} else if (seg_kind[q] == KIND_NATIVE) {"),
+    "replica_slot_of_rank_zero": ("off[q] = (d * B + seg_wslot[q]) * W;", "off[q] = seg_wslot[q] * W;"),
 }
 
 

@@ -653,3 +653,61 @@ def test_prefetch_all_tokens_on_one_expert():
     after = oracle.prefetch_weight(c, t, w, np.zeros((R, 2, 8), np.uint16))
     assert np.array_equal(after[1:, 0], np.broadcast_to(w[0], (R - 1, 8)))
     assert not after[0].any() and not after[1:, 1].any()
+
+
+# ------------------------------------------------------- segment weights ---
+
+
+def test_segment_weights_worked_example():
+    """The worked example by hand (R=2, E=4, S=3, K=2): rank 0 holds experts 0 and 1
+    natively; rank 1 holds 2 and 3 and the overflow of expert 1 as a replica piece in
+    weight slot 0.  With W = 5: native segments read home rows e * 5, the piece reads
+    replica slot (rank 1 * budget 2 + slot 0) * 5; the remaining entries read nothing."""
+    c = cfg(2, 4, 2, 3, budget=2)
+    idx = np.array([[[0, 1], [0, 1], [1, 2]], [[0, 1], [0, 3], [1, 2]]], np.int32)
+    _, t = oracle.plan(c, idx)
+    buf, off = oracle.segment_weights(c, t, 5)
+    assert buf.tolist() == [[0, 0, -1, -1], [0, 0, 1, -1]]
+    assert off.tolist() == [[0, 5, -1, -1], [10, 15, 10, -1]]
+    # past the budget (budget 0) the piece is remote: it reads the home expert's row
+    c0 = cfg(2, 4, 2, 3, budget=0, mode=1)
+    _, t0 = oracle.plan(c0, idx)
+    buf0, off0 = oracle.segment_weights(c0, t0, 5)
+    assert buf0[1, 2] == 0 and off0[1, 2] == 1 * 5
+
+
+@pytest.mark.parametrize("case", [(8, 64, 8, 96, 8, 20.0, 0), (8, 64, 8, 96, 2, 20.0, 1),
+                                  (4, 32, 4, 50, 0, 5.0, 1), (3, 9, 3, 40, 3, 3.0, 0)])
+def test_segment_weights_against_piece_tables(case):
+    """Derived from the piece list and the replica-slot table instead of the segment
+    table: each local piece reads slot (rank * budget + slot) and that slot holds the
+    piece's expert; each remote piece and each native expert reads the home row; every
+    rank has exactly n_seg entries that read something."""
+    R, E, K, S, B, mv, mode = case
+    c = cfg(R, E, K, S, budget=B, mode=mode)
+    idx, _, _ = make_routing(R, E, K, S, mv, seed=31)
+    st, t = oracle.plan(c, idx)
+    W = 7
+    buf, off = oracle.segment_weights(c, t, W)
+    L = E // R
+    expect = {}  # (rank, expert) -> (buf, off)
+    for d in range(R):
+        for i in range(L):
+            expect[(d, d * L + i)] = (0, (d * L + i) * W)
+    n_piece = int(t["n_piece"][0])
+    for p in range(n_piece):
+        d, e, j = int(t["piece_rank"][p]), int(t["piece_expert"][p]), int(t["piece_wslot"][p])
+        if j >= 0:
+            assert t["rep_expert"][d * B + j] == e
+            expect[(d, e)] = (1, (d * B + j) * W)
+        else:
+            expect[(d, e)] = (0, e * W)
+    got = {}
+    for d in range(R):
+        for i in range(E):
+            if buf[d, i] >= 0:
+                got[(d, int(t["seg_expert"][d, i]))] = (int(buf[d, i]), int(off[d, i]))
+            else:
+                assert off[d, i] == -1
+        assert (buf[d] >= 0).sum() == t["n_seg"][d]
+    assert got == expect
