@@ -11,6 +11,7 @@
  *   moonep_reduce_grad       fold replica-expert gradients into their home experts
  *   moonep_dispatch_backward gradient of dispatch (sum of a token's K slot gradients)
  *   moonep_prefetch_weight   copy duplicated experts' weights into replica slots
+ *   moonep_segment_weights   the weight matrix each segment's expert computation reads
  *   moonep_fused_forward     plan + dispatch + combine of the identity expert in one launch
  *
  * Conventions shared by every call:
@@ -269,6 +270,27 @@ MOONEP_API moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
 MOONEP_API moonep_status_t moonep_prefetch_weight(const moonep_config_t *cfg,
                                                   const void *plan_arena, const uint16_t *weights,
                                                   uint16_t *rep_weights, int64_t W,
+                                                  int32_t *dev_status, moonep_stream_t stream);
+
+/* The weights each entry of the plan's segment tables computes with, for the expert
+ * computation between dispatch and combine (same page, replica-slot paragraph: a
+ * duplicated expert runs on its receiving rank with the weights prefetched into a
+ * local slot, and past the slot budget reads them on its home rank).  Entry
+ * q = d*E + i of rank d's segment table gets:
+ *   MOONEP_SEG_REPLICA  rep_weights + (d*budget + seg_wslot[q]) * W
+ *   MOONEP_SEG_NATIVE   weights + seg_expert[q] * W
+ *   MOONEP_SEG_REMOTE   weights + seg_expert[q] * W  (the home copy, read remotely)
+ *   unused              NULL
+ * Written on the device (no host read of the plan), so a grouped expert kernel can
+ * take the rows [seg_start, seg_start + seg_len) of each segment and this pointer.
+ *   weights      device bf16 [E, W] (home expert weights; only addresses are formed)
+ *   rep_weights  device bf16 [R, budget, W] (may be NULL when budget == 0)
+ *   seg_weights  device, R*E pointers, 8-byte aligned; written
+ * An entry naming an expert or a slot out of range is NULL and sets
+ * MOONEP_DEV_BAD_PLAN. */
+MOONEP_API moonep_status_t moonep_segment_weights(const moonep_config_t *cfg, const void *plan_arena,
+                                                  const uint16_t *weights, const uint16_t *rep_weights,
+                                                  int64_t W, const uint16_t **seg_weights,
                                                   int32_t *dev_status, moonep_stream_t stream);
 
 /* The zero_copy=False comparison path ("MoonshotAI/MoonEP 딥다이브" §6: the

@@ -98,6 +98,14 @@ def test_null_and_misaligned_pointers_rejected_on_host():
     assert L.moonep_prefetch_weight(cp, base, base, base, 0, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_dispatch_via_buffer(cp, base, base, None, base, base, base, 0) == \
         me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base, None, base, 16, base, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base, base, None, 16, base, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base, base, base, 0, base, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base, base, base, 16, None, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base, base, base, 16, base + 4, base, 0) == \
+        me.ERR_INVALID_ARG
+    assert L.moonep_segment_weights(cp, base + 16, base, base, 16, base, base, 0) == \
+        me.ERR_INVALID_ARG
     assert L.moonep_combine_via_buffer(cp, base, base, base, None, base, base, base, 0) == \
         me.ERR_INVALID_ARG
     c13 = me.Config(R=2, E=4, K=2, S=3, H=13, budget=2)  # rows not 16-byte multiples

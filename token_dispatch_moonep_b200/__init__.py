@@ -136,6 +136,8 @@ _lib.moonep_dispatch_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_dispatch_backward.restype = _ST
 _lib.moonep_prefetch_weight.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
 _lib.moonep_prefetch_weight.restype = _ST
+_lib.moonep_segment_weights.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP, _VP]
+_lib.moonep_segment_weights.restype = _ST
 _lib.moonep_dispatch_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_dispatch_via_buffer.restype = _ST
 _lib.moonep_combine_via_buffer.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]
@@ -278,6 +280,16 @@ def moonep_prefetch_weight(cfg: Config, plan_arena, weights, rep_weights, W: int
     _check("moonep_prefetch_weight", _lib.moonep_prefetch_weight(
         ctypes.byref(cfg), _ptr(plan_arena), _ptr(weights), _ptr(rep_weights), int(W),
         _ptr(dev_status), _stream(stream)))
+
+
+def moonep_segment_weights(cfg: Config, plan_arena, weights, rep_weights, W: int, seg_weights,
+                           dev_status, stream=None) -> None:
+    """Device pointers [R*E] (an int64 tensor) to the weight matrix of every segment-table
+    entry: replica pieces their local slot, native segments and remote pieces the home
+    expert's row, unused entries 0 (see include/moonep.h)."""
+    _check("moonep_segment_weights", _lib.moonep_segment_weights(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(weights), _ptr(rep_weights), int(W),
+        _ptr(seg_weights), _ptr(dev_status), _stream(stream)))
 
 
 def moonep_dispatch_via_buffer(cfg: Config, plan_arena, x, comm, comm_index, recv, dev_status,
