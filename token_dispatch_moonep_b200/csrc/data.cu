@@ -5,8 +5,9 @@
 // involved.
 //
 // Rows are moved as 16-byte vectors (8 bf16).  A warp owns a token (dispatch:
-// half a row of one; combine-backward: two warps per token): lane k (< K)
-// holds the token's k-th slot and gate and broadcasts them with shuffles.
+// half a row of one; combine: half a row when the batch is small;
+// combine-backward: two warps per token): lane k (< K) holds the token's k-th
+// slot and gate and broadcasts them with shuffles.
 // reduce_grad streams through shared memory with bulk asynchronous copies.
 // Rows whose byte length or base address is not 16-byte aligned take a scalar
 // (one bf16 per lane) path.

@@ -929,18 +929,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_multichunk_kernel(PlanArgs 
 }
 
 // ============================================ one chunk per CTA, every CTA solves ===
-// plan_kernel: W CTAs, CTA k owns chunk k (W = number of chunks, all co-resident).
-//   count    stable ranks of the chunk's pairs and its histogram (count_chunk);
-//            the histogram is published with an arrival flag.
-//   gather   every CTA sums every chunk's histogram: the expert counts, and the
-//            counts of the chunks before its own (its pairs' base offsets).  A
-//            chunk is added as soon as its flag shows this launch's epoch.
-//   solve    every CTA solves the O(E + R) balance problem itself, in one warp
-//            (shuffle scans and shared memory, no block barriers).  All CTAs
-//            reach the same tables, so no CTA waits for another after the gather.
-//   place    each CTA places its own pairs straight from its shared memory.
-//   tables   each CTA writes its share of the user-facing plan tables.
-// One grid-wide exchange (the arrivals) per plan.
+// plan_kernel (phases at the top of this file): its shared-memory state.  One
+// grid-wide exchange (the arrivals) per plan; every CTA then holds the whole solve.
 struct FastSmem {
   int *cnt, *base, *gcst, *kept, *ovf, *oend, *nst, *row0, *npc, *i0, *pid0, *eflag, *epos;  // [E]
   int *load, *over, *def, *ridx, *ntot, *nseg, *rrank, *rbase, *rend, *rfirst, *rlast;  // [R]
