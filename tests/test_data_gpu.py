@@ -229,6 +229,34 @@ def test_reduce_grad_gradient_equivalence_exact():
     assert np.array_equal(bf16_bits_to_f32(got).astype(np.int64), ref)
 
 
+def test_reduce_grad_overlapping_calls_share_one_plan():
+    """Two gradient matrices of one plan folded on two streams at once (the data calls
+    only read the plan arena): both results exact."""
+    import torch
+    import token_dispatch_moonep_b200 as me
+    R, E, K, S, B, P = 8, 256, 8, 256, 32, 16384
+    cfg, ocfg, ot, arena = _setup(R, E, K, S, 8, mv=20.0, seed=44, budget=B, mode=1)
+    assert int(ot["n_piece"][0]) > 0
+    mats = [(normal_bf16((R, B, P), seed=44 + j, stream=11), normal_bf16((E, P), seed=44 + j, stream=12))
+            for j in range(2)]
+    dev = [(to_dev(r), to_dev(h)) for r, h in mats]
+    statuses = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    torch.cuda.synchronize()
+    for _ in range(3):  # three rounds: the replicas are added three times
+        for j in range(2):
+            with torch.cuda.stream(streams[j]):
+                me.moonep_reduce_grad(cfg, arena, dev[j][0], dev[j][1], P, statuses[j],
+                                      streams[j].cuda_stream)
+    torch.cuda.synchronize()
+    for j in range(2):
+        assert int(statuses[j].item()) == 0
+        rep, ref = mats[j]
+        for _ in range(3):
+            ref = oracle.reduce_grad(ocfg, ot, rep, ref)
+        _exact(to_np(dev[j][1]), ref)
+
+
 def test_reduce_grad_without_budget_is_a_no_op():
     cfg, ocfg, ot, arena = _setup(4, 16, 2, 40, 8, mv=4.0, seed=9, budget=0, mode=1)
     home = integer_bf16((16, 16), seed=9)
