@@ -27,6 +27,10 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
 * ``reduce_grad`` — with integer-valued bf16 gradients all fp32 sums are
   exact, so home + replicas must equal, bit for bit, the no-replication
   gradient (§4 pattern 3, §8 exercise E).
+* ``reduce_grad_f32`` — the same fold over fp32 gradient buffers.  Pinned by the
+  no-replication identity with integers past bf16's exact range (so a rounding
+  through bf16 fails), and by the order of the fp32 additions: home first, then
+  the pieces in ascending receiver, fixed by sums whose result depends on it.
 * ``dispatch_backward`` — the adjoint of dispatch: with integer-valued data
   <dispatch(x), dR> = <x, dispatch_backward(dR)> exactly, and
   dispatch_backward(dispatch(x)) = K*x.
@@ -108,6 +112,8 @@ def _L():
         lib.orc_combine_backward_tokens.restype = None
         lib.orc_reduce_grad.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
         lib.orc_reduce_grad.restype = None
+        lib.orc_reduce_grad_f32.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
+        lib.orc_reduce_grad_f32.restype = None
         lib.orc_dispatch_backward_tokens.argtypes = [cp, vp, vp, vp, ctypes.c_int64, vp]
         lib.orc_dispatch_backward_tokens.restype = None
         lib.orc_prefetch_weight.argtypes = [cp, vp, vp, vp, ctypes.c_int32, vp, vp, ctypes.c_int64]
@@ -217,6 +223,20 @@ def reduce_grad(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray, hom
     pr = _c(tables["piece_rank"], np.int32)
     pw = _c(tables["piece_wslot"], np.int32)
     _L().orc_reduce_grad(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(rep), _p(home), P)
+    return home
+
+
+def reduce_grad_f32(cfg: Config, tables: Dict[str, np.ndarray], rep: np.ndarray,
+                    home: np.ndarray) -> np.ndarray:
+    """New fp32 home gradients [E, P] (a copy); ``rep`` is fp32 [R, budget, P]: the
+    replica pieces added into their home expert in fp32, in plan order."""
+    home = np.array(home, dtype=np.float32, copy=True, order="C")
+    rep = _c(rep, np.float32)
+    P = home.shape[-1]
+    pe = _c(tables["piece_expert"], np.int32)
+    pr = _c(tables["piece_rank"], np.int32)
+    pw = _c(tables["piece_wslot"], np.int32)
+    _L().orc_reduce_grad_f32(ctypes.byref(cfg), _p(pe), _p(pr), _p(pw), len(pe), _p(rep), _p(home), P)
     return home
 
 

@@ -47,6 +47,8 @@
  *              dgate[t,k] = sum_h dOut[t,h] * y[slot_k,h] accumulated in double
  *   reduce_grad home[e] = bf16(float(home[e]) + sum over e's local replica pieces,
  *              in O order (ascending receiver), of float(rep[d][slot]))
+ *   reduce_grad over fp32 gradient buffers: the same sum in the same order, with
+ *              fp32 gradients in and out (no bf16 rounding anywhere)
  *   dispatch-bw dx[t] = bf16( sum_k float(dRecv[slot_k]) ), fp32 adds in k order (the
  *              adjoint of dispatch; the backward pass reuses the forward plan, §4 pattern 1)
  *   prefetch   rep_w[d][j] = w[e] for every local replica piece (d, j) of expert e
@@ -384,6 +386,29 @@ void orc_reduce_grad(const orc_config *c, const int32_t *piece_expert, const int
         acc = acc + orc_bf16_to_f32(rep[slot * P + q]);
       }
       home[e * P + q] = orc_f32_to_bf16(acc);
+    }
+  }
+}
+
+/* For every expert e with a local replica piece, over fp32 gradient buffers:
+   home[e] = home[e] + the pieces' gradients, fp32 additions starting from home[e]
+   and taking the pieces in O order (ascending receiver), with no rounding to bf16
+   ("MoonshotAI/MoonEP 딥다이브" §4 pattern 3: replica gradients are added into
+   the home expert's gradient; a training step that keeps its expert gradients in
+   fp32 buffers folds them there).  rep is [R, budget, P], home [E, P]. */
+void orc_reduce_grad_f32(const orc_config *c, const int32_t *piece_expert, const int32_t *piece_rank,
+                         const int32_t *piece_wslot, int32_t n_piece, const float *rep, float *home,
+                         int64_t P) {
+  const int64_t B = c->budget;
+  for (int64_t e = 0; e < c->E; e++) {
+    for (int64_t q = 0; q < P; q++) {
+      float acc = home[e * P + q];
+      for (int32_t i = 0; i < n_piece; i++) {
+        if (piece_expert[i] != e || piece_wslot[i] < 0) continue;
+        int64_t slot = (int64_t)piece_rank[i] * B + piece_wslot[i];
+        acc = acc + rep[slot * P + q];
+      }
+      home[e * P + q] = acc;
     }
   }
 }

@@ -711,3 +711,77 @@ def test_segment_weights_against_piece_tables(case):
                 assert off[d, i] == -1
         assert (buf[d] >= 0).sum() == t["n_seg"][d]
     assert got == expect
+
+
+# ------------------------------------------------------- reduce_grad, fp32 ---
+
+
+@pytest.mark.parametrize("case", [(8, 32, 4, 64, 4, 6.0), (8, 64, 8, 32, 8, 15.0)])
+def test_reduce_grad_f32_equals_no_replication(case):
+    """The fp32 fold reproduces the no-replication gradient exactly with integer
+    gradients up to a few thousand: exact in fp32 but not in bf16 (integers past 256
+    round there), so a fold that rounds through bf16 anywhere fails."""
+    R, E, K, S, B, mv = case
+    idx, _, _ = make_routing(R, E, K, S, mv, seed=18)
+    c = cfg(R, E, K, S, budget=B)
+    st, t = oracle.plan(c, idx)
+    assert st == oracle.OK and int(t["n_piece"][0]) > 0
+    P = 16
+    NvS = int(t["nvs"][0])
+    g = np.random.default_rng(18).integers(-300, 301, size=(R * NvS, P)).astype(np.int64)
+    ref = np.zeros((E, P), np.int64)
+    np.add.at(ref, idx.ravel(), g[t["slot_of"]])
+    home = np.zeros((E, P), np.int64)
+    rep = np.zeros((R, B, P), np.int64)
+    L = E // R
+    for d in range(R):
+        for i in range(int(t["n_seg"][d])):
+            e, s0, ln = t["seg_expert"][d, i], t["seg_start"][d, i], t["seg_len"][d, i]
+            part = g[d * NvS + s0: d * NvS + s0 + ln].sum(0)
+            if i < L:
+                home[e] += part
+            else:
+                rep[d, t["seg_wslot"][d, i]] += part
+    assert np.abs(ref).max() > 256 and np.abs(ref).max() < 2 ** 24  # beyond bf16, exact in fp32
+    new = oracle.reduce_grad_f32(c, t, rep.astype(np.float32), home.astype(np.float32))
+    assert new.dtype == np.float32
+    assert np.array_equal(new.astype(np.int64), ref)
+
+
+def test_reduce_grad_f32_adds_home_first_then_pieces_by_rank():
+    """All tokens on expert 0 of 3 ranks: its overflow is one piece on rank 1 and one on
+    rank 2.  home = 1, rank 1's piece = 1, rank 2's = 2**24: ((1 + 1) + 2**24) = 2**24 + 2
+    exactly, while the other orders lose a 1 to rounding (2**24 + 1 is not an fp32)."""
+    R, E, K, S, B = 3, 3, 1, 4, 1
+    c = cfg(R, E, K, S, budget=B)
+    idx = np.zeros((R, S, K), np.int32)
+    st, t = oracle.plan(c, idx)
+    n = int(t["n_piece"][0])
+    pe, pr, pw = t["piece_expert"][:n], t["piece_rank"][:n], t["piece_wslot"][:n]
+    assert list(pe) == [0, 0] and list(pr) == [1, 2] and list(pw) == [0, 0]
+    P = 2
+    home = np.zeros((E, P), np.float32)
+    home[0] = 1.0
+    rep = np.zeros((R, B, P), np.float32)
+    rep[1, 0] = 1.0
+    rep[2, 0] = 2.0 ** 24
+    new = oracle.reduce_grad_f32(c, t, rep, home)
+    assert (new[0] == np.float32(2.0 ** 24 + 2)).all()
+    assert np.float32(np.float32(1.0 + 2.0 ** 24) + 1.0) == np.float32(2.0 ** 24)  # the other orders
+    assert (new[1:] == 0).all()
+
+
+def test_reduce_grad_f32_leaves_unreplicated_experts_alone():
+    R, E, K, S, B = 4, 16, 2, 30, 2
+    idx, _, _ = make_routing(R, E, K, S, 4.0, seed=9)
+    c = cfg(R, E, K, S, budget=B)
+    st, t = oracle.plan(c, idx)
+    P = 10
+    rng = np.random.default_rng(19)
+    home = rng.standard_normal((E, P)).astype(np.float32)
+    rep = rng.standard_normal((R, B, P)).astype(np.float32)
+    new = oracle.reduce_grad_f32(c, t, rep, home)
+    touched = np.zeros(E, bool)
+    touched[t["piece_expert"][t["piece_wslot"] >= 0]] = True
+    assert touched.any() and not touched.all()
+    assert np.array_equal(new[~touched], home[~touched])
