@@ -13,7 +13,9 @@ kernels / their CUDA-event time, plus plan µs per layer.  ms_per_step comes fro
 K steps with events only around them (kernels overlap their launch gaps as in
 use); the per-kernel times, the metric and the roofline from a second pass of
 K steps with an event after every kernel; `b2b_ms` per data kernel from ten
-launches in a row between two events (no event between launches).
+launches in a row between two events (no event between launches).  Training
+workloads also report `reduce_grad_f32`: the same fold over fp32 gradient buffers
+on the step's plan (not part of the step), timed the same two ways.
 Default workload: R=8 ranks, E=256 experts, K=8, S=4096 tokens/rank, H=7168,
 maxvio 0.2, replica budget 32 (training).  The default run then adds, on the
 same line: `sweep` — the forward layer (plan + dispatch + combine) of the same
@@ -383,6 +385,41 @@ def time_back_to_back(layer, n=10, ops=None):
         torch.cuda.synchronize()
         out[name] = e0.elapsed_time(e1) / n
     return out
+
+
+def time_reduce_grad_f32(layer, n=10):
+    """reduce_grad over fp32 gradient buffers (moonep_reduce_grad_f32; not one of the
+    step's kernels: the step folds bf16 gradients) on the step's plan and row length:
+    its launch time with events around each launch and launched n times back to back,
+    against its algorithmic bytes (the bf16 fold's, at 4 bytes a value)."""
+    torch, me, w = layer.torch, layer.me, layer.w
+    g = torch.Generator(device=layer.dev).manual_seed(7)
+    rep = torch.randn(w.R * w.budget * layer.P, generator=g, device=layer.dev)
+    home = torch.randn(w.E * layer.P, generator=g, device=layer.dev)
+    fn = lambda: me.moonep_reduce_grad_f32(layer.cfg, layer.arena, rep, home, layer.P, layer.status)
+    fn()
+    fn()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    each = []
+    for _ in range(n):
+        e0, e1 = ev(), ev()
+        e0.record()
+        fn()
+        e1.record()
+        each.append((e0, e1))
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(c) for a, c in each) / n
+    b2b = e0.elapsed_time(e1) / n
+    nbytes = 2 * layer.bytes()["reduce_grad"]
+    del rep, home
+    torch.cuda.empty_cache()
+    return {"ms": ms, "b2b_ms": b2b, "bytes": nbytes, "GBs": nbytes / (ms * 1e-3) / 1e9,
+            "b2b_GBs": nbytes / (b2b * 1e-3) / 1e9}
 
 
 def host_cost(layer, n=500):
@@ -926,6 +963,14 @@ def main():
     replicas = {"pieces": layer.n_piece, "local": layer.n_local, "remote": layer.n_remote,
                 "experts_replicated": layer.n_rep_exp}
 
+    rg_f32 = None
+    if layer.train and not args.no_extra:
+        rg_f32 = time_reduce_grad_f32(layer)
+        rg_f32["ms"], rg_f32["b2b_ms"] = max_over_ranks(pg, [rg_f32["ms"], rg_f32["b2b_ms"]], device)
+        for k in ("", "b2b_"):
+            rg_f32[k + "GBs"] = rg_f32["bytes"] / (rg_f32[k + "ms"] * 1e-3) / 1e9
+            rg_f32[k + "frac"] = rg_f32[k + "GBs"] / peak
+
     e2e = None
     if not args.no_e2e:
         n = min(args.steps, 20)
@@ -961,6 +1006,7 @@ def main():
             "plan_us_per_layer": kern["plan"]["ms"] * 1e3,
             "layer_us": 1e3 * (kern["plan"]["ms"] + kern["dispatch"]["ms"] + kern["combine"]["ms"]),
             "kernels": kern,
+            "reduce_grad_f32": rg_f32,
             "replicas": replicas,
             "device_status": st,
             "roofline": roof,

@@ -9,6 +9,7 @@
  *   moonep_combine           gate-weighted gather-sum of expert outputs back to tokens
  *   moonep_combine_backward  gradients of combine w.r.t. expert outputs and gates
  *   moonep_reduce_grad       fold replica-expert gradients into their home experts
+ *                            (moonep_reduce_grad_f32: the same over fp32 gradient buffers)
  *   moonep_dispatch_backward gradient of dispatch (sum of a token's K slot gradients)
  *   moonep_prefetch_weight   copy duplicated experts' weights into replica slots
  *   moonep_segment_weights   the weight matrix each segment's expert computation reads
@@ -246,6 +247,19 @@ MOONEP_API moonep_status_t moonep_combine_backward(const moonep_config_t *cfg, c
 MOONEP_API moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
                                    const uint16_t *rep_grads, uint16_t *home_grads, int64_t P,
                                    int32_t *dev_status, moonep_stream_t stream);
+
+/* reduce_grad over fp32 gradient buffers (the same section of the deep-dive page; for
+ * a training step that keeps its expert gradients in fp32):
+ *   for each expert e with local replica pieces (plan order = ascending rank d):
+ *     home[e, :] = home[e, :] + sum_d rep[d, wslot_d(e), :]
+ * fp32 additions starting from home[e, :], pieces in that order, in place; no bf16
+ * rounding anywhere.  rep_grads device fp32 [R, budget, P]; home_grads device fp32
+ * [E, P]; P >= 1.  Rows are staged in shared memory by bulk copies when P % 4 == 0
+ * and both buffers are 16-byte aligned, else a scalar kernel does the same sums.
+ * Arguments, errors and dev_status bits as for moonep_reduce_grad. */
+MOONEP_API moonep_status_t moonep_reduce_grad_f32(const moonep_config_t *cfg, const void *plan_arena,
+                                       const float *rep_grads, float *home_grads, int64_t P,
+                                       int32_t *dev_status, moonep_stream_t stream);
 
 /* Backward of dispatch (reuses the forward plan, "MoonshotAI/MoonEP 딥다이브" §4
  * pattern 1): the gradient of each token row is the sum of the gradients of

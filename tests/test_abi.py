@@ -90,6 +90,11 @@ def test_null_and_misaligned_pointers_rejected_on_host():
         me.ERR_INVALID_ARG
     assert L.moonep_reduce_grad(cp, base, base, base, 0, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_reduce_grad(cp, base, None, base, 16, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_reduce_grad_f32(cp, base, base, base, 0, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_reduce_grad_f32(cp, base, None, base, 16, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_reduce_grad_f32(cp, base, base, None, 16, base, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_reduce_grad_f32(cp, base, base, base, 16, None, 0) == me.ERR_INVALID_ARG
+    assert L.moonep_reduce_grad_f32(cp, base + 16, base, base, 16, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_plan_view(cp, None, ctypes.byref(me.PlanView())) == me.ERR_INVALID_ARG
     assert L.moonep_dispatch_backward(cp, base, None, base, base, 0) == me.ERR_INVALID_ARG
     assert L.moonep_dispatch_backward(cp, base, base, None, base, 0) == me.ERR_INVALID_ARG

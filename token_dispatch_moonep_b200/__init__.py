@@ -16,6 +16,7 @@ The functions keep the C names::
     moonep_combine(cfg, plan_arena, y, gates, out, dev_status, stream=None)
     moonep_combine_backward(cfg, plan_arena, dout, y, gates, dy, dgates, dev_status, stream=None)
     moonep_reduce_grad(cfg, plan_arena, rep_grads, home_grads, P, dev_status, stream=None)
+    moonep_reduce_grad_f32(cfg, plan_arena, rep_grads, home_grads, P, dev_status, stream=None)
     moonep_dispatch_backward(cfg, plan_arena, d_recv, dx, dev_status, stream=None)
     moonep_prefetch_weight(cfg, plan_arena, weights, rep_weights, W, dev_status, stream=None)
     moonep_dispatch_via_buffer(cfg, plan_arena, x, comm, comm_index, recv, dev_status, stream=None)
@@ -132,6 +133,8 @@ _lib.moonep_combine_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
 _lib.moonep_combine_backward.restype = _ST
 _lib.moonep_reduce_grad.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
 _lib.moonep_reduce_grad.restype = _ST
+_lib.moonep_reduce_grad_f32.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
+_lib.moonep_reduce_grad_f32.restype = _ST
 _lib.moonep_dispatch_backward.argtypes = [_CP, _VP, _VP, _VP, _VP, _VP]
 _lib.moonep_dispatch_backward.restype = _ST
 _lib.moonep_prefetch_weight.argtypes = [_CP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]
@@ -265,6 +268,14 @@ def moonep_combine_backward(cfg: Config, plan_arena, dout, y, gates, dy, dgates,
 def moonep_reduce_grad(cfg: Config, plan_arena, rep_grads, home_grads, P: int, dev_status,
                        stream=None) -> None:
     _check("moonep_reduce_grad", _lib.moonep_reduce_grad(
+        ctypes.byref(cfg), _ptr(plan_arena), _ptr(rep_grads), _ptr(home_grads), int(P),
+        _ptr(dev_status), _stream(stream)))
+
+
+def moonep_reduce_grad_f32(cfg: Config, plan_arena, rep_grads, home_grads, P: int, dev_status,
+                           stream=None) -> None:
+    """reduce_grad over fp32 gradient buffers (float32 tensors [R, budget, P] and [E, P])."""
+    _check("moonep_reduce_grad_f32", _lib.moonep_reduce_grad_f32(
         ctypes.byref(cfg), _ptr(plan_arena), _ptr(rep_grads), _ptr(home_grads), int(P),
         _ptr(dev_status), _stream(stream)))
 

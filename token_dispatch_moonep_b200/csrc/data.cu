@@ -8,9 +8,9 @@
 // half a row of one; combine: half a row when the batch is small;
 // combine-backward: two warps per token): lane k (< K) holds the token's k-th
 // slot and gate and broadcasts them with shuffles.
-// reduce_grad streams through shared memory with bulk asynchronous copies.
-// Rows whose byte length or base address is not 16-byte aligned take a scalar
-// (one bf16 per lane) path.
+// reduce_grad (over bf16 or fp32 gradient rows) streams through shared memory
+// with bulk asynchronous copies.  Rows whose byte length or base address is not
+// 16-byte aligned take a scalar (one value per lane) path.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -479,7 +479,8 @@ combine_bwd_scalar_kernel(const int32_t *__restrict__ slot_of, const uint16_t *_
 // chunks, each further stage the next four.  One producer thread per CTA
 // issues cp.async.bulk copies (completion counted in bytes on the stage's
 // mbarrier); eight consumer warps add the stage's rows in fp32 in piece order
-// and, after the unit's last stage, store the bf16 result over the home chunk.
+// and, after the unit's last stage, store the result over the home chunk (bf16
+// gradients: rounded once to bf16; fp32 gradient buffers: the fp32 sum itself).
 // Three stages of four chunks per CTA and two CTAs per SM keep up to 192 KB
 // per SM in flight with no registers held for it (measured against 4 stages
 // of 3 chunks: equal at 10 pieces over 6 experts, 6% faster at 59 over 54).
@@ -565,10 +566,14 @@ __device__ __forceinline__ bool local_piece(const Tables &t, int pc, int *row) {
 }
 }  // namespace rg
 
+// kF32: fp32 gradient rows (4 values per 16-byte vector) instead of bf16 (8); the
+// sums are the same fp32 additions in the same order, with no rounding to bf16.
+template <bool kF32>
 __global__ void __launch_bounds__(rg::kThreadsRg, 1)
 reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__restrict__ home,
                         int64_t nvec, int32_t *status) {
   using namespace rg;
+  constexpr int kEl = kF32 ? 4 : 8;  // values per 16-byte vector
   pdl_wait();
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
@@ -669,7 +674,7 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
     const int64_t off = (u % nch) * kChunk;
     const int64_t nv = (rowbytes - off < kChunk ? rowbytes - off : kChunk) / 16;
     const int ng = stages_of(nl, kSlots);
-    float acc[kVecPerLane][8];
+    float acc[kVecPerLane][kEl];
     int left = nl;
     for (int g = 0; g < ng; g++, k++) {
       const int s = (int)(k % kStages);
@@ -687,8 +692,12 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
           const uint32_t wd[4] = {h.x, h.y, h.z, h.w};
 #pragma unroll
           for (int w = 0; w < 4; w++) {
-            acc[j][2 * w] = bf16_lo(wd[w]);
-            acc[j][2 * w + 1] = bf16_hi(wd[w]);
+            if constexpr (kF32) {
+              acc[j][w] = __uint_as_float(wd[w]);
+            } else {
+              acc[j][2 * w] = bf16_lo(wd[w]);
+              acc[j][2 * w + 1] = bf16_hi(wd[w]);
+            }
           }
         }
         q = 1;
@@ -705,8 +714,12 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
           const uint32_t wd[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
           for (int w = 0; w < 4; w++) {
-            acc[j][2 * w] = __fadd_rn(acc[j][2 * w], bf16_lo(wd[w]));
-            acc[j][2 * w + 1] = __fadd_rn(acc[j][2 * w + 1], bf16_hi(wd[w]));
+            if constexpr (kF32) {
+              acc[j][w] = __fadd_rn(acc[j][w], __uint_as_float(wd[w]));
+            } else {
+              acc[j][2 * w] = __fadd_rn(acc[j][2 * w], bf16_lo(wd[w]));
+              acc[j][2 * w + 1] = __fadd_rn(acc[j][2 * w + 1], bf16_hi(wd[w]));
+            }
           }
         }
       }
@@ -720,10 +733,15 @@ reduce_grad_bulk_kernel(rg::Tables t, const uint4 *__restrict__ rep, uint4 *__re
       const int64_t v = (warp * kVecPerLane + j) * 32 + lane;
       if (v < nv) {
         uint4 o;
-        o.x = pack_bf16x2(acc[j][0], acc[j][1]);
-        o.y = pack_bf16x2(acc[j][2], acc[j][3]);
-        o.z = pack_bf16x2(acc[j][4], acc[j][5]);
-        o.w = pack_bf16x2(acc[j][6], acc[j][7]);
+        if constexpr (kF32) {
+          o = make_uint4(__float_as_uint(acc[j][0]), __float_as_uint(acc[j][1]),
+                         __float_as_uint(acc[j][2]), __float_as_uint(acc[j][3]));
+        } else {
+          o.x = pack_bf16x2(acc[j][0], acc[j][1]);
+          o.y = pack_bf16x2(acc[j][2], acc[j][3]);
+          o.z = pack_bf16x2(acc[j][4], acc[j][5]);
+          o.w = pack_bf16x2(acc[j][6], acc[j][7]);
+        }
         hrow[v] = o;
       }
     }
@@ -905,11 +923,20 @@ prefetch_weight_scalar_kernel(const int32_t *__restrict__ replicated, const int3
   }
 }
 
+// reduce_grad's scalar path (rows not in whole aligned 16-byte vectors): one value of
+// a replicated expert's row per thread, the same fp32 additions in piece order.
+// Gradient values of either type read as fp32 and stored back in their own type.
+__device__ __forceinline__ float grad_to_f(uint16_t b) { return bf16_to_f(b); }
+__device__ __forceinline__ float grad_to_f(float v) { return v; }
+__device__ __forceinline__ void grad_store(uint16_t *p, float v) { *p = f_to_bf16(v); }
+__device__ __forceinline__ void grad_store(float *p, float v) { *p = v; }
+
+template <class T>
 __global__ void __launch_bounds__(kThreads)
 reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t *__restrict__ scalars,
                           const int32_t *__restrict__ pbeg, const int32_t *__restrict__ pend,
                           const int32_t *__restrict__ prank, const int32_t *__restrict__ pwslot,
-                          const uint16_t *__restrict__ rep, uint16_t *__restrict__ home, int64_t P,
+                          const T *__restrict__ rep, T *__restrict__ home, int64_t P,
                           int R, int E, int B, int PMAX, int32_t *status) {
   pdl_wait();
   int64_t n_exp = scalars[S_N_REPLICATED];
@@ -927,7 +954,7 @@ reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t 
       set_status(status, MOONEP_DEV_BAD_PLAN);
       continue;
     }
-    float acc = bf16_to_f(home[(int64_t)e * P + c]);
+    float acc = grad_to_f(home[(int64_t)e * P + c]);
     for (int pc = b; pc < en; pc++) {
       const int ws = pwslot[pc], rk = prank[pc];
       if (ws < 0) continue;
@@ -935,17 +962,19 @@ reduce_grad_scalar_kernel(const int32_t *__restrict__ replicated, const int32_t 
         set_status(status, MOONEP_DEV_BAD_PLAN);
         continue;
       }
-      acc = __fadd_rn(acc, bf16_to_f(rep[((int64_t)rk * B + ws) * P + c]));
+      acc = __fadd_rn(acc, grad_to_f(rep[((int64_t)rk * B + ws) * P + c]));
     }
-    home[(int64_t)e * P + c] = f_to_bf16(acc);
+    grad_store(home + (int64_t)e * P + c, acc);
   }
 }
 
 int num_sms() { return current_sm_count(); }
 
-// Co-resident CTAs per SM of reduce_grad_bulk_kernel, -1 on a CUDA error.  Its shared
-// memory limit is a per-context function attribute: it is raised once per CUDA context
-// and the occupancy answer is kept with the context id, per device.
+// Co-resident CTAs per SM of reduce_grad_bulk_kernel<kF32>, -1 on a CUDA error.  Its
+// shared memory limit is a per-context function attribute: it is raised once per CUDA
+// context and the occupancy answer is kept with the context id, per device and per
+// instantiation.
+template <bool kF32>
 int rg_blocks_per_sm() {
   static std::mutex mu;
   static unsigned long long ctx_of[kMaxDevices];
@@ -959,9 +988,9 @@ int rg_blocks_per_sm() {
   std::lock_guard<std::mutex> lk(mu);
   if (ctx != 0 && ctx_of[dev] == ctx && per_sm_of[dev] > 0) return per_sm_of[dev];
   int per_sm = 0;
-  if (cudaFuncSetAttribute(reduce_grad_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(reduce_grad_bulk_kernel<kF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            rg::kSmem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_grad_bulk_kernel, rg::kThreadsRg,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reduce_grad_bulk_kernel<kF32>, rg::kThreadsRg,
                                                     rg::kSmem) != cudaSuccess || per_sm < 1) {
     cudaGetLastError();
     return -1;
@@ -1082,10 +1111,15 @@ extern "C" moonep_status_t moonep_combine_backward(const moonep_config_t *cfg,
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
 }
 
-extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
-                                              const uint16_t *rep_grads, uint16_t *home_grads,
-                                              int64_t P_elems, int32_t *dev_status,
-                                              moonep_stream_t stream) {
+namespace {
+// reduce_grad over gradient rows of T (bf16 bits or fp32): the bulk-copy pipeline when
+// rows are whole 16-byte vectors at 16-byte aligned bases, else the scalar kernel.
+template <class T>
+moonep_status_t reduce_grad_impl(const moonep_config_t *cfg, const void *plan_arena, const T *rep_grads,
+                                 T *home_grads, int64_t P_elems, int32_t *dev_status,
+                                 moonep_stream_t stream) {
+  constexpr bool kF32 = sizeof(T) == 4;
+  constexpr int64_t kPerVec = 16 / sizeof(T);
   Dims d;
   if (!make_dims(cfg, &d) || !plan_arena || !dev_status || P_elems < 1)
     return MOONEP_ERR_INVALID_ARG;
@@ -1094,24 +1128,38 @@ extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const 
   if (d.B == 0) return MOONEP_OK;  // no replica slots, nothing to fold
   PlanPtrs P = plan_ptrs(d, plan_arena);
   cudaStream_t st = to_cuda(stream);
-  if (P_elems % 8 == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
-    // bulk copies need 16-byte aligned rows: P % 8 == 0 and aligned bases
-    const int per_sm = rg_blocks_per_sm();
+  if (P_elems % kPerVec == 0 && aligned16(rep_grads) && aligned16(home_grads)) {
+    const int per_sm = rg_blocks_per_sm<kF32>();
     if (per_sm < 1) return MOONEP_ERR_CUDA;
     const rg::Tables t{P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN],
                        P.f[F_EXP_PIECE_END], P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT],
                        (int)d.R, (int)d.E, (int)d.B, (int)d.PMAX, debug_wait_limit_ns(),
                        debug_phantom() > 0 ? 16 * debug_phantom() : 0};
-    launch(reduce_grad_bulk_kernel, (unsigned)(num_sms() * per_sm), rg::kThreadsRg, rg::kSmem, st,
+    launch(reduce_grad_bulk_kernel<kF32>, (unsigned)(num_sms() * per_sm), rg::kThreadsRg, rg::kSmem, st,
         t, reinterpret_cast<const uint4 *>(rep_grads), reinterpret_cast<uint4 *>(home_grads),
-        P_elems / 8, dev_status);
+        P_elems / kPerVec, dev_status);
   } else {
-    launch(reduce_grad_scalar_kernel, (unsigned)num_sms() * 8, kThreads, 0, st,
+    launch(reduce_grad_scalar_kernel<T>, (unsigned)num_sms() * 8, kThreads, 0, st,
         P.f[F_REPLICATED], P.f[F_SCALARS], P.f[F_EXP_PIECE_BEGIN], P.f[F_EXP_PIECE_END],
         P.f[F_PIECE_RANK], P.f[F_PIECE_WSLOT], rep_grads, home_grads, P_elems, (int)d.R,
         (int)d.E, (int)d.B, (int)d.PMAX, dev_status);
   }
   return cudaGetLastError() == cudaSuccess ? MOONEP_OK : MOONEP_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" moonep_status_t moonep_reduce_grad(const moonep_config_t *cfg, const void *plan_arena,
+                                              const uint16_t *rep_grads, uint16_t *home_grads,
+                                              int64_t P_elems, int32_t *dev_status,
+                                              moonep_stream_t stream) {
+  return reduce_grad_impl(cfg, plan_arena, rep_grads, home_grads, P_elems, dev_status, stream);
+}
+
+extern "C" moonep_status_t moonep_reduce_grad_f32(const moonep_config_t *cfg, const void *plan_arena,
+                                                  const float *rep_grads, float *home_grads,
+                                                  int64_t P_elems, int32_t *dev_status,
+                                                  moonep_stream_t stream) {
+  return reduce_grad_impl(cfg, plan_arena, rep_grads, home_grads, P_elems, dev_status, stream);
 }
 
 extern "C" moonep_status_t moonep_dispatch_backward(const moonep_config_t *cfg,
