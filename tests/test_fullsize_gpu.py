@@ -12,7 +12,8 @@ both sides compute with the same operations in the same order (fused
 multiply-adds in ascending k, one product, fp32 additions in ascending k or in
 piece order), so they must be bit-identical too; the 1e-3 norm-relative bar of
 the contract is asserted beside it.  dgate is an fp32 dot product on the GPU
-and an fp64 one in the oracle: 1e-3 norm-relative.
+and an fp64 one in the oracle: 1e-3 norm-relative.  reduce_grad over fp32
+gradient buffers is the same fp32 additions with no rounding: bit-identical.
 """
 import numpy as np
 import pytest
@@ -171,3 +172,22 @@ def test_full_size_layer(name, mv, seed):
     touched[ot["piece_expert"][ot["piece_wslot"] >= 0]] = True
     assert touched.any()
     assert np.array_equal(got_home[~touched], home_cols[~touched])  # untouched experts unchanged
+
+    # ---- the same fold over fp32 gradient buffers (the pool's rows as fp32)
+    del rep, home
+    torch.cuda.empty_cache()
+    pool32 = bf16_bits_to_f32(pool)
+    pool32_d = torch.from_numpy(pool32).to(dev)
+    rep32 = pool32_d[torch.from_numpy(rep_map).to(dev)]     # [R*B, P] fp32
+    home32 = pool32_d[torch.from_numpy(home_map).to(dev)]   # [E, P] fp32
+    me.moonep_reduce_grad_f32(cfg, arena, rep32, home32, P, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref32 = oracle.reduce_grad_f32(ocfg, ot, pool32[rep_map][:, cols].reshape(R, B, len(cols)),
+                                   pool32[home_map][:, cols])
+    got32 = home32[:, torch.from_numpy(cols).to(dev)].cpu().numpy()
+    assert float(np.abs(got32.astype(np.float64) - ref32).max()) <= TOL * float(np.abs(ref32).max())
+    assert np.array_equal(got32.view(np.uint32), ref32.view(np.uint32)), int((got32 != ref32).sum())
+    assert np.array_equal(got32[~touched], pool32[home_map][:, cols][~touched])
+    del rep32, home32, pool32_d
+    torch.cuda.empty_cache()
