@@ -21,19 +21,21 @@ What each function follows, and what pins it (the ``-m "not gpu"`` tests):
 * ``dispatch`` — the bit-copy definition (§2② zero copy); pinned by the
   round trip and the "every row written exactly once" poison check.
 * ``combine`` — fp32 gate-weighted sum (§3③ combine); pinned against the fp64
-  closed form sum_k w_k x within the bf16 + fp32 rounding bound (§8 exercise C).
+  closed form sum_k w_k x within the bf16 + fp32 rounding bound (§8 exercise C),
+  and its order (ascending k) by three terms whose fp32 sum depends on it.
 * ``combine_backward`` — per-element closed forms: dY = w*dOut within half a bf16
   ulp of the fp64 product; dgate = <dOut, x> for the identity expert, in fp64.
 * ``reduce_grad`` — with integer-valued bf16 gradients all fp32 sums are
   exact, so home + replicas must equal, bit for bit, the no-replication
-  gradient (§4 pattern 3, §8 exercise E).
+  gradient (§4 pattern 3, §8 exercise E); its order (home first, then the
+  pieces by ascending receiving rank) by three terms whose sum depends on it.
 * ``reduce_grad_f32`` — the same fold over fp32 gradient buffers.  Pinned by the
   no-replication identity with integers past bf16's exact range (so a rounding
   through bf16 fails), and by the order of the fp32 additions: home first, then
   the pieces in ascending receiver, fixed by sums whose result depends on it.
 * ``dispatch_backward`` — the adjoint of dispatch: with integer-valued data
   <dispatch(x), dR> = <x, dispatch_backward(dR)> exactly, and
-  dispatch_backward(dispatch(x)) = K*x.
+  dispatch_backward(dispatch(x)) = K*x; its order (ascending k) as combine's.
 * ``prefetch_weight`` — every local replica slot holds its expert's weights
   bit for bit, every other slot is untouched; closed form for all tokens on
   one expert.

@@ -6,7 +6,8 @@ slot, a dropped term, a missing gate, a skipped replica, ignored alignment,
 truncating instead of rounding, reversed per-expert order, a half dot
 product, a remote piece or a replica slot mapped to the wrong weights, an fp32
 fold that rounds through bf16, adds its pieces in the wrong order or adds the
-home gradient last),
+home gradient last, a combine, dispatch-backward or bf16 fold that adds its
+terms in the wrong order),
 builds it with gcc, and runs the pin tests against it: at least one
 pin must fail.  Everything runs on the CPU.
 """
@@ -45,6 +46,20 @@ MUTANTS = {
     "remote_piece_reads_replica_slot": ("} else if (seg_kind[q] == KIND_NATIVE || seg_kind[q] == KIND_REMOTE) {",
                                         "} else if (seg_kind[q] == KIND_NATIVE) {"),
     "replica_slot_of_rank_zero": ("off[q] = (d * B + seg_wslot[q]) * W;", "off[q] = seg_wslot[q] * W;"),
+    "combine_k_descending": ("      for (int64_t k = 0; k < K; k++) {\n        int64_t row = slot_of[t * K + k];\n"
+                             "        acc = fmaf(",
+                             "      for (int64_t k = K - 1; k >= 0; k--) {\n        int64_t row = slot_of[t * K + k];\n"
+                             "        acc = fmaf("),
+    "dispatch_backward_k_descending": ("      for (int64_t k = 0; k < K; k++) {\n        int64_t row = slot_of[t * K + k];\n"
+                                       "        acc = acc + orc_bf16_to_f32(drecv",
+                                       "      for (int64_t k = K - 1; k >= 0; k--) {\n        int64_t row = slot_of[t * K + k];\n"
+                                       "        acc = acc + orc_bf16_to_f32(drecv"),
+    "reduce_pieces_descending": ("for (int32_t i = 0; i < n_piece; i++) {\n        if (piece_expert[i] != e"
+                                 " || piece_wslot[i] < 0) continue;\n        int64_t slot = (int64_t)"
+                                 "piece_rank[i] * B + piece_wslot[i];\n        acc = acc + orc_bf16_to_f32(rep[",
+                                 "for (int32_t i = n_piece - 1; i >= 0; i--) {\n        if (piece_expert[i] != e"
+                                 " || piece_wslot[i] < 0) continue;\n        int64_t slot = (int64_t)"
+                                 "piece_rank[i] * B + piece_wslot[i];\n        acc = acc + orc_bf16_to_f32(rep["),
     "reduce_f32_rounds_through_bf16": ("      home[e * P + q] = acc;",
                                        "      home[e * P + q] = orc_bf16_to_f32(orc_f32_to_bf16(acc));"),
     "reduce_f32_pieces_descending": ("for (int32_t i = 0; i < n_piece; i++) {\n        if (piece_expert[i] != e"

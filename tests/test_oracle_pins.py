@@ -785,3 +785,51 @@ def test_reduce_grad_f32_leaves_unreplicated_experts_alone():
     touched[t["piece_expert"][t["piece_wslot"] >= 0]] = True
     assert touched.any() and not touched.all()
     assert np.array_equal(new[~touched], home[~touched])
+
+
+# ------------------------------------------ the order of the fp32 additions ---
+# Three terms 2**24, 1, -2**24 (each exact in bf16): added in that order they give 0,
+# because 2**24 + 1 rounds back to 2**24 in fp32; in any other order the 1 survives.
+# So these pin the order each fold takes (the reading: ascending k for a token's
+# slots, the home gradient first and then the pieces by ascending receiving rank),
+# which the rounding bounds and the integer identities above do not see.
+_ORDERED = np.array([2.0 ** 24, 1.0, -(2.0 ** 24)], np.float32)
+
+
+def test_combine_accumulates_in_ascending_k():
+    c = cfg(1, 3, 3, 1, H=2, budget=0)
+    slot_of = np.array([0, 1, 2], np.int32)
+    y = f32_to_bf16_bits(np.repeat(_ORDERED[:, None], 2, axis=1))
+    out = oracle.combine(c, slot_of, y, np.ones(3, np.float32))
+    assert (bf16_bits_to_f32(out) == 0.0).all()
+    rev = oracle.combine(c, slot_of[::-1].copy(), y, np.ones(3, np.float32))
+    assert (bf16_bits_to_f32(rev) == 1.0).all()  # the same three rows in the other order
+
+
+def test_dispatch_backward_adds_in_ascending_k():
+    c = cfg(1, 3, 3, 1, H=2, budget=0)
+    slot_of = np.array([0, 1, 2], np.int32)
+    drecv = f32_to_bf16_bits(np.repeat(_ORDERED[:, None], 2, axis=1))
+    assert (bf16_bits_to_f32(oracle.dispatch_backward(c, slot_of, drecv)) == 0.0).all()
+    rev = oracle.dispatch_backward(c, slot_of[::-1].copy(), drecv)
+    assert (bf16_bits_to_f32(rev) == 1.0).all()
+
+
+def test_reduce_grad_adds_home_first_then_pieces_by_rank():
+    """All tokens on expert 0 of 3 ranks: its overflow is one piece on rank 1 and one on
+    rank 2.  home = 2**24, rank 1's piece 1, rank 2's piece -2**24 fold to 0."""
+    R, E, K, S, B = 3, 3, 1, 4, 1
+    c = cfg(R, E, K, S, budget=B)
+    st, t = oracle.plan(c, np.zeros((R, S, K), np.int32))
+    n = int(t["n_piece"][0])
+    assert list(t["piece_expert"][:n]) == [0, 0] and list(t["piece_rank"][:n]) == [1, 2]
+    P = 2
+    home = np.zeros((E, P), np.float32)
+    home[0] = _ORDERED[0]
+    rep = np.zeros((R, B, P), np.float32)
+    rep[1, 0] = _ORDERED[1]
+    rep[2, 0] = _ORDERED[2]
+    new = oracle.reduce_grad(c, t, f32_to_bf16_bits(rep), f32_to_bf16_bits(home))
+    assert (bf16_bits_to_f32(new) == 0.0).all()
+    new32 = oracle.reduce_grad_f32(c, t, rep, home)
+    assert (new32 == 0.0).all()
