@@ -833,3 +833,45 @@ def test_reduce_grad_adds_home_first_then_pieces_by_rank():
     assert (bf16_bits_to_f32(new) == 0.0).all()
     new32 = oracle.reduce_grad_f32(c, t, rep, home)
     assert (new32 == 0.0).all()
+
+
+@settings(max_examples=120, deadline=None, derandomize=True)
+@given(R=hs.integers(1, 8), L=hs.integers(1, 4), K=hs.integers(1, 8), S=hs.integers(1, 40),
+       budget_frac=hs.floats(0, 1), mode=hs.integers(0, 1), align=hs.sampled_from([1, 2, 4]),
+       alpha=hs.floats(0, 3), seed=hs.integers(0, 2**31 - 1))
+def test_reduce_grad_folds_property(R, L, K, S, budget_frac, mode, align, alpha, seed):
+    """Both folds over drawn plans, REMOTE pieces included.  Each buffer row carries an
+    integer gradient; home rows sum a rank's native segments, replica slots their local
+    pieces.  After the fold every expert holds the gradient of all its pairs except the
+    rows of its REMOTE pieces (they have no replica slot and add nothing)."""
+    E = R * L
+    K = min(K, E)
+    B = int(round(budget_frac * L))
+    p = (np.arange(E) + 1.0) ** -alpha
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(E, size=(R, S, K), p=p / p.sum()).astype(np.int32)
+    c = cfg(R, E, K, S, budget=B, mode=mode, align=align)
+    st, t = oracle.plan(c, idx)
+    assert st in (oracle.OK, oracle.BUDGET)
+    NvS, P = int(t["nvs"][0]), 3
+    g = rng.integers(-2, 3, size=(R * NvS, P)).astype(np.int64)
+    want = np.zeros((E, P), np.int64)
+    np.add.at(want, idx.ravel(), g[t["slot_of"]])  # no replication: all of e's pairs
+    home = np.zeros((E, P), np.int64)
+    rep = np.zeros((R, max(B, 1), P), np.int64)
+    for d in range(R):
+        for i in range(int(t["n_seg"][d])):
+            e, s0, ln = t["seg_expert"][d, i], t["seg_start"][d, i], t["seg_len"][d, i]
+            part = g[d * NvS + s0: d * NvS + s0 + ln].sum(0)
+            if i < L:
+                home[e] += part
+            elif t["seg_wslot"][d, i] >= 0:
+                rep[d, t["seg_wslot"][d, i]] += part
+            else:
+                want[e] -= part  # a REMOTE piece: its rows are not folded
+    got32 = oracle.reduce_grad_f32(c, t, rep[:, :B].astype(np.float32), home.astype(np.float32))
+    assert np.array_equal(got32.astype(np.int64), want)
+    if max(np.abs(want).max(), np.abs(home).max(), np.abs(rep).max()) <= 256:  # exact in bf16
+        to_bf16 = lambda a: f32_to_bf16_bits(a.astype(np.float32))
+        got = oracle.reduce_grad(c, t, to_bf16(rep[:, :B]), to_bf16(home))
+        assert np.array_equal(bf16_bits_to_f32(got).astype(np.int64), want)
