@@ -875,3 +875,42 @@ def test_reduce_grad_folds_property(R, L, K, S, budget_frac, mode, align, alpha,
         to_bf16 = lambda a: f32_to_bf16_bits(a.astype(np.float32))
         got = oracle.reduce_grad(c, t, to_bf16(rep[:, :B]), to_bf16(home))
         assert np.array_equal(bf16_bits_to_f32(got).astype(np.int64), want)
+
+
+@settings(max_examples=100, deadline=None, derandomize=True)
+@given(R=hs.integers(1, 8), L=hs.integers(1, 4), K=hs.integers(1, 8), S=hs.integers(1, 40),
+       budget_frac=hs.floats(0, 1), mode=hs.integers(0, 1), alpha=hs.floats(0, 3),
+       seed=hs.integers(0, 2**31 - 1))
+def test_replica_weights_property(R, L, K, S, budget_frac, mode, alpha, seed):
+    """prefetch_weight and segment_weights over drawn plans, REMOTE pieces included:
+    every local piece's slot holds its expert's row and every other slot is untouched;
+    every segment reads its replica slot (local piece) or the home row (native segment,
+    REMOTE piece), derived here from the piece list rather than the segment table."""
+    E = R * L
+    K = min(K, E)
+    B = int(round(budget_frac * L))
+    p = (np.arange(E) + 1.0) ** -alpha
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(E, size=(R, S, K), p=p / p.sum()).astype(np.int32)
+    c = cfg(R, E, K, S, budget=B, mode=mode)
+    st, t = oracle.plan(c, idx)
+    W = 5
+    w = rng.integers(0, 1 << 16, size=(E, W)).astype(np.uint16)
+    before = rng.integers(0, 1 << 16, size=(R, B, W)).astype(np.uint16)
+    after = oracle.prefetch_weight(c, t, w, before)
+    n = int(t["n_piece"][0])
+    pe, pr, pw = t["piece_expert"][:n], t["piece_rank"][:n], t["piece_wslot"][:n]
+    filled = np.zeros((R, B), bool)
+    expect = {(d, d * L + i): (0, (d * L + i) * W) for d in range(R) for i in range(L)}
+    for e, d, j in zip(pe, pr, pw):
+        if j >= 0:
+            assert np.array_equal(after[d, j], w[e])
+            filled[d, j] = True
+            expect[(int(d), int(e))] = (1, (int(d) * B + int(j)) * W)
+        else:
+            expect[(int(d), int(e))] = (0, int(e) * W)
+    assert np.array_equal(after[~filled], before[~filled])
+    buf, off = oracle.segment_weights(c, t, W)
+    got = {(d, int(t["seg_expert"][d, i])): (int(buf[d, i]), int(off[d, i]))
+           for d in range(R) for i in range(E) if buf[d, i] >= 0}
+    assert got == expect
