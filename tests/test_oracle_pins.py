@@ -914,3 +914,39 @@ def test_replica_weights_property(R, L, K, S, budget_frac, mode, alpha, seed):
     got = {(d, int(t["seg_expert"][d, i])): (int(buf[d, i]), int(off[d, i]))
            for d in range(R) for i in range(E) if buf[d, i] >= 0}
     assert got == expect
+
+
+@settings(max_examples=100, deadline=None, derandomize=True)
+@given(R=hs.integers(1, 8), L=hs.integers(1, 4), K=hs.integers(1, 8), S=hs.integers(1, 40),
+       budget_frac=hs.floats(0, 1), mode=hs.integers(0, 1), align=hs.sampled_from([1, 2, 4, 16]),
+       alpha=hs.floats(0, 3), seed=hs.integers(0, 2**31 - 1))
+def test_data_path_property(R, L, K, S, budget_frac, mode, align, alpha, seed):
+    """dispatch, the identity expert's combine and dispatch-backward over drawn plans
+    (repeated experts in a token, padding rows, REMOTE pieces): every valid row is its
+    source token's row and padding rows keep what was there; combine equals sum_k w_k x
+    within the bf16 + fp32 rounding bound; dispatch-backward of dispatch is K x exactly
+    on small integers (§8 exercise C; the adjoint of dispatch)."""
+    E = R * L
+    K = min(K, E)
+    B = int(round(budget_frac * L))
+    p = (np.arange(E) + 1.0) ** -alpha
+    rng = np.random.default_rng(seed)
+    idx = rng.choice(E, size=(R, S, K), p=p / p.sum()).astype(np.int32)
+    c = cfg(R, E, K, S, H=4, budget=B, mode=mode, align=align)
+    st, t = oracle.plan(c, idx)
+    T, H, NvS = R * S, 4, int(t["nvs"][0])
+    x = f32_to_bf16_bits(rng.standard_normal((T, H)).astype(np.float32))
+    poison = np.full((R * NvS, H), 0xFFC1, np.uint16)
+    recv = oracle.dispatch(c, t["slot_of"], x, poison.copy())
+    valid = t["slot_src"] >= 0
+    assert np.array_equal(recv[valid], x[t["slot_src"][valid] // K])
+    assert (recv[~valid] == 0xFFC1).all()
+    z = rng.standard_normal((T, K))
+    w = (np.exp(z) / np.exp(z).sum(1, keepdims=True)).astype(np.float32)
+    out = oracle.combine(c, t["slot_of"], recv, w)
+    exact = w.astype(np.float64).sum(1, keepdims=True) * bf16_bits_to_f32(x).astype(np.float64)
+    bound = _bf16_half_ulp(exact) * (1 + 2 ** -7) + K * 2.0 ** -24 * np.abs(exact) * 2
+    assert (np.abs(bf16_bits_to_f32(out).astype(np.float64) - exact) <= bound).all()
+    xi = f32_to_bf16_bits(rng.integers(-16, 17, size=(T, H)).astype(np.float32))
+    dx = oracle.dispatch_backward(c, t["slot_of"], oracle.dispatch(c, t["slot_of"], xi))
+    assert np.array_equal(bf16_bits_to_f32(dx), K * bf16_bits_to_f32(xi))
