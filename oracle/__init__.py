@@ -5,7 +5,11 @@ leg may import this package.  It wraps the plain C implementation in
 ``moonep_oracle.c`` (built with gcc, strict IEEE arithmetic, no fast-math) and
 shares nothing with the CUDA library: no code, header, table or constant.
 
-What each function follows, and what pins it (the ``-m "not gpu"`` tests):
+What each function follows, and what pins it (the ``-m "not gpu"`` tests).
+Besides the pins below, property tests draw small plans (1-8 ranks, budgets
+0..L, both modes, padding, repeated experts in a token, REMOTE pieces) and
+check on each the plan's invariants, the data path, the two gradient folds
+and the replica-weight tables:
 
 * ``plan`` — the pages fix the outcome: every rank receives exactly S*K
   token-slots ("Moonshot AI Open-Sources MoonEP", S x K paragraph), overloaded
