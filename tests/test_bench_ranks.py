@@ -145,3 +145,10 @@ def test_profiles_name_the_current_sources():
         parts = dict(kv.split("=", 1) for kv in ln.split())
         assert now[parts["source"]] == parts["sha"]
         assert now["moonep_internal.cuh"] == parts["header_sha"]
+    # bench.py's own reader finds a current line for each of the step's seven kernels,
+    # so the headline run's roofline carries the measured traffic
+    import bench
+    got = bench.ncu_traffic(bench.DEFAULT_WORKLOAD, 0.2, 0)
+    assert set(got) == {"plan", "prefetch", "dispatch", "combine", "combine_bwd", "dispatch_bwd",
+                        "reduce_grad"}, sorted(got)
+    assert all(v > 0 for v in got.values())
