@@ -29,6 +29,11 @@
  *     zeroes it once and reads it whenever it chooses.
  *   - bf16 tensors are passed as uint16_t bit patterns, row-major, rows
  *     contiguous.  Row counts use the symbols of moonep_config_t.
+ *   - Alignment: every pointer is aligned to its element type, as C requires
+ *     of a typed pointer (2 bytes for bf16, 4 for int32 and fp32).  The calls
+ *     check null pointers and the 256-byte alignment of the plan arena and the
+ *     workspace.  Rows whose byte length or base is not a multiple of 16 take a
+ *     scalar path.  Element alignment itself is not checked.
  *   - Layouts: topk_idx int32 [R, S, K]; gates fp32 [R, S, K]; x / out / dout
  *     bf16 [R, S, H]; the dispatch buffer bf16 [R, NvS, H] (rank d owns rows
  *     d*NvS .. d*NvS+NvS-1); replica gradients bf16 [R, budget, P]; home
